@@ -1,0 +1,226 @@
+// api.cu - host side of the C ABI: argument validation, workspace layout, status word, launches.
+//
+// Nothing here allocates or frees device memory, and nothing synchronises except
+// entmax_attn_check(). Every argument error returns before the first CUDA call.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "entmax_attn.h"
+#include "fwd_common.cuh"
+#include "launch.h"
+
+namespace eattn {
+
+__device__ int g_status;  // ENTMAX_OK, or the first device-side error since the last check
+
+namespace {
+
+// A kernel that waits on a barrier nobody arrives at, bounded by limit_ns: exercises the timeout path.
+__global__ void selftest_timeout_kernel(uint64_t limit_ns, int* status) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint64_t t0 = globaltimer();
+        bool ok = false;
+        for (uint32_t i = 0; i < kWaitIterCap; ++i) {
+            if (mbar_try_wait(&bar, 0)) { ok = true; break; }
+            if ((i & 31u) == 31u && globaltimer() - t0 > limit_ns) break;
+        }
+        if (!ok) atomicExch(status, (int)ENTMAX_ERR_TIMEOUT);
+        mbar_arrive(&bar);  // complete the phase so the barrier is left in a clean state
+    }
+}
+
+int* status_ptr() {
+    static int* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<int*>(p);
+    }
+    return cache[dev];
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Dims {
+    int B, H, n, d, mb, nqb, nkb, nw, nwq, bins, ntiles;
+};
+
+entmax_status check_dims(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* o, Dims* out) {
+    if (B < 1 || H < 1 || n < 1 || d < 1) return ENTMAX_ERR_INVALID;
+    if ((long long)B * H > (1ll << 30) || (long long)n > (1ll << 30)) return ENTMAX_ERR_INVALID;
+    if (dt != ENTMAX_BF16 && dt != ENTMAX_FP32) return ENTMAX_ERR_INVALID;
+    if (d != 64 && d != 128) return ENTMAX_ERR_UNSUPPORTED;
+    const int mb = (o && o->mask_block) ? o->mask_block : 64;
+    if (mb != 32 && mb != 64) return ENTMAX_ERR_UNSUPPORTED;
+    if (dt == ENTMAX_BF16 && mb != 64) return ENTMAX_ERR_UNSUPPORTED;
+    const int bins = (o && o->hist_bins) ? o->hist_bins : 256;
+    if (bins != 64 && bins != 128 && bins != 256) return ENTMAX_ERR_UNSUPPORTED;
+    if (o && (o->init_mode < 0 || o->init_mode > 1)) return ENTMAX_ERR_INVALID;
+    if (o && o->scale != 0.0f && !(o->scale > 0.0f && isfinite(o->scale))) return ENTMAX_ERR_INVALID;
+    Dims D;
+    D.B = B; D.H = H; D.n = n; D.d = d; D.mb = mb; D.bins = bins;
+    D.nqb = (n + mb - 1) / mb;
+    D.nkb = (n + mb - 1) / mb;
+    D.nw = (D.nkb + 31) / 32;
+    D.nwq = (D.nqb + 31) / 32;
+    D.ntiles = (n + kTileRows - 1) / kTileRows;
+    *out = D;
+    return ENTMAX_OK;
+}
+
+struct Workspace {
+    float* obar;
+    float* sum_u;
+    float* delta;
+    uint32_t* maskT;
+    size_t bytes;
+};
+
+Workspace layout(const Dims& D, void* base) {
+    const size_t rows = (size_t)D.B * D.H * D.n;
+    Workspace w;
+    char* p = static_cast<char*>(base);
+    size_t off = 0;
+    w.obar = reinterpret_cast<float*>(p + off);
+    off = align256(off + rows * D.d * sizeof(float));
+    w.sum_u = reinterpret_cast<float*>(p + off);
+    off = align256(off + rows * sizeof(float));
+    w.delta = reinterpret_cast<float*>(p + off);
+    off = align256(off + rows * sizeof(float));
+    w.maskT = reinterpret_cast<uint32_t*>(p + off);
+    off = align256(off + (size_t)D.B * D.H * D.nkb * D.nwq * sizeof(uint32_t));
+    w.bytes = off;
+    return w;
+}
+
+entmax_status check_workspace(const Dims& D, const entmax_opts* o, Workspace* w) {
+    if (!o || !o->workspace) return ENTMAX_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(o->workspace) & 255u) != 0) return ENTMAX_ERR_ALIGN;
+    *w = layout(D, o->workspace);
+    if (o->workspace_bytes < w->bytes) return ENTMAX_ERR_WORKSPACE;
+    return ENTMAX_OK;
+}
+
+inline entmax_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ENTMAX_OK : ENTMAX_ERR_CUDA; }
+
+}  // namespace
+}  // namespace eattn
+
+using namespace eattn;
+
+#define EATTN_API __attribute__((visibility("default")))
+
+extern "C" {
+
+EATTN_API int entmax_attn_version(void) { return 1; }
+
+EATTN_API const char* entmax_status_str(entmax_status s) {
+    switch (s) {
+        case ENTMAX_OK: return "ok";
+        case ENTMAX_ERR_INVALID: return "invalid argument";
+        case ENTMAX_ERR_UNSUPPORTED: return "unsupported configuration";
+        case ENTMAX_ERR_ALIGN: return "pointer not aligned (16 bytes for tensors, 256 for the workspace)";
+        case ENTMAX_ERR_CUDA: return "CUDA error";
+        case ENTMAX_ERR_TIMEOUT: return "device-side wait timed out";
+        case ENTMAX_ERR_WORKSPACE: return "workspace missing or too small";
+    }
+    return "unknown status";
+}
+
+EATTN_API size_t entmax_attn_workspace_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts) {
+    Dims D;
+    if (check_dims(B, H, n, d, dt, opts, &D) != ENTMAX_OK) return 0;
+    return layout(D, nullptr).bytes;
+}
+
+EATTN_API entmax_status entmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* tau,
+                              uint32_t* block_mask, int B, int H, int n, int d, float alpha, int causal,
+                              entmax_dtype dt, const entmax_opts* opts, void* stream) {
+    if (!Q || !K || !V || !O || !tau || !block_mask) return ENTMAX_ERR_INVALID;
+    if (!(alpha > 1.0f) || !isfinite(alpha) || (causal != 0 && causal != 1)) return ENTMAX_ERR_INVALID;
+    Dims D;
+    entmax_status st = check_dims(B, H, n, d, dt, opts, &D);
+    if (st != ENTMAX_OK) return st;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return ENTMAX_ERR_ALIGN;
+    Workspace ws;
+    if ((st = check_workspace(D, opts, &ws)) != ENTMAX_OK) return st;
+    int* status = status_ptr();
+    if (!status) return ENTMAX_ERR_CUDA;
+
+    FwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.Q = Q; a.K = K; a.V = V; a.O = O; a.tau = tau; a.mask = block_mask;
+    a.obar = ws.obar; a.sum_u = ws.sum_u;
+    a.tau_hist = opts->tau_hist; a.steps = opts->steps; a.stats = opts->stats; a.status = status;
+    a.B = B; a.H = H; a.n = n; a.d = d;
+    a.nqb = D.nqb; a.nkb = D.nkb; a.nw = D.nw; a.mb = D.mb; a.causal = causal; a.ntiles = D.ntiles;
+    const float scale = opts->scale != 0.0f ? opts->scale : 1.0f / sqrtf((float)d);
+    a.sp = make_solve_params(alpha, scale, D.bins, opts->init_mode);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+    cudaError_t e;
+    if (dt == ENTMAX_FP32) {
+        e = launch_fwd_simt(a, true, s);
+    } else {
+        e = launch_fwd_tc(a, s);
+        if (e == cudaSuccess) e = launch_mask_transpose(block_mask, ws.maskT, B * H, D.nqb, D.nkb, D.nw, D.nwq, s);
+    }
+    return from_cuda(e);
+}
+
+EATTN_API entmax_status entmax_attn_check(void* stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return ENTMAX_ERR_CUDA;
+    int* p = status_ptr();
+    if (!p) return ENTMAX_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ENTMAX_ERR_CUDA;
+    if (v != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return ENTMAX_ERR_CUDA;
+    }
+    return static_cast<entmax_status>(v);
+}
+
+EATTN_API entmax_status entmax_attn_selftest_timeout(int limit_us, void* stream) {
+    if (limit_us < 1 || limit_us > 2000000) return ENTMAX_ERR_INVALID;
+    int* status = status_ptr();
+    if (!status) return ENTMAX_ERR_CUDA;
+    selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((uint64_t)limit_us * 1000ull, status);
+    return from_cuda(cudaGetLastError());
+}
+
+}  // extern "C"
+
+// ---- entry points whose kernels are added in later files (placeholders until then) ----
+extern "C" {
+EATTN_API entmax_status entmax_attn_bwd(const void*, const void*, const void*, const void*, const void*,
+                                        const float*, const uint32_t*, void*, void*, void*, int, int, int, int,
+                                        float, int, entmax_dtype, const entmax_opts*, void*) {
+    return ENTMAX_ERR_UNSUPPORTED;
+}
+EATTN_API entmax_status softmax_attn_fwd(const void*, const void*, const void*, void*, float*, int, int, int, int,
+                                         int, entmax_dtype, const entmax_opts*, void*) {
+    return ENTMAX_ERR_UNSUPPORTED;
+}
+EATTN_API entmax_status softmax_attn_bwd(const void*, const void*, const void*, const void*, const void*,
+                                         const float*, void*, void*, void*, int, int, int, int, int, entmax_dtype,
+                                         const entmax_opts*, void*) {
+    return ENTMAX_ERR_UNSUPPORTED;
+}
+}

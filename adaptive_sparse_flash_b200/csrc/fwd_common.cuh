@@ -1,0 +1,58 @@
+// fwd_common.cuh - argument block and sweep schedule shared by the two forward kernels.
+#pragma once
+
+#include <stdint.h>
+
+#include "entmax_attn.h"
+#include "entmax_row.cuh"
+
+namespace eattn {
+
+struct FwdArgs {
+    const void* Q;
+    const void* K;
+    const void* V;
+    void* O;
+    float* tau;
+    uint32_t* mask;    // [B,H,nqb,nw]
+    float* obar;       // workspace: U V, fp32 [B,H,n,d]
+    float* sum_u;      // workspace: fp32 [B,H,n]
+    float* tau_hist;   // optional
+    uint8_t* steps;    // optional
+    entmax_stats* stats;
+    int* status;
+    int B, H, n, d;
+    int nqb, nkb, nw;  // mask query blocks, key blocks (of mb), words per mask row
+    int mb;            // mask block
+    int causal;
+    int ntiles;        // 128-row query tiles per head
+    SolveParams sp;
+};
+
+enum SweepKind : int { kSweepDense = 0, kSweepRefine = 1, kSweepPV = 2, kSweepDone = 3 };
+
+// Number of allowed keys of query row `row`.
+__device__ __forceinline__ int allowed_keys(int row, int n, int causal) {
+    return causal ? min(row + 1, n) : n;
+}
+
+// Per-CTA statistics, reduced into entmax_stats at the end of a tile.
+struct TileStats {
+    uint32_t rows, steps, fallbacks, candidate_blocks, nonzero_blocks, causal_blocks, sweeps;
+    uint32_t step_hist[kMaxSteps + 1];
+};
+
+__device__ __forceinline__ void flush_stats(entmax_stats* g, const TileStats& t) {
+    if (!g) return;
+    atomicAdd(&g->rows, (unsigned long long)t.rows);
+    atomicAdd(&g->steps, (unsigned long long)t.steps);
+    atomicAdd(&g->fallbacks, (unsigned long long)t.fallbacks);
+    atomicAdd(&g->candidate_blocks, (unsigned long long)t.candidate_blocks);
+    atomicAdd(&g->nonzero_blocks, (unsigned long long)t.nonzero_blocks);
+    atomicAdd(&g->causal_blocks, (unsigned long long)t.causal_blocks);
+    atomicAdd(&g->sweeps, (unsigned long long)t.sweeps);
+    for (int i = 0; i <= kMaxSteps; ++i)
+        if (t.step_hist[i]) atomicAdd(&g->step_hist[i], (unsigned long long)t.step_hist[i]);
+}
+
+}  // namespace eattn

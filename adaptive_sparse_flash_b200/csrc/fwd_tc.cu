@@ -1,0 +1,648 @@
+// fwd_tc.cu - alpha-entmax attention forward for bf16 on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+// One CTA per (b, h, 128-row query tile), 192 threads:
+//   warps 0-3  compute: thread r owns query row r of the tile and TMEM lane r (tcgen05.ld 32x32b);
+//   warp 4     MMA issue (one thread): S = Q K^T into TMEM, O += P V and U V into TMEM;
+//   warp 5     TMA issue (one thread): Q once, K (and V in P V sweeps) blocks of 64 keys into a ring.
+// TMEM columns: S double buffer [0, 64) and [64, 128), O [128, 128 + D), U V [128 + D, 128 + 2D).
+//
+// The key blocks of a tile are swept several times; before each sweep the compute warps publish a
+// plan (sweep kind + bit set of key blocks) that the two issuing warps follow:
+//   dense  - every causal key block: running max, left-edge histogram (shared memory, one ring of
+//            B slots per row), candidate blocks with an entry above max - 1;
+//   refine - candidate blocks only: solver sums at the current tau, one hybrid-solver update;
+//   P V    - candidate blocks: p = [z - tau]_+^k and u = [z - tau]_+^(k-1) rounded to bf16 into
+//            shared memory (128B-swizzled, K-major) for the P V and U V MMAs; exact block mask; the
+//            sums check sum p = 1 and the sweep repeats while any row's tau still moved.
+// (AdaSplash-2, gist.science (de), section 2: histogram initialisation, hybrid solver, bit-packed
+// block mask, only nonzero blocks processed; the histogram lives in on-chip memory, O(B) per row.)
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "fwd_common.cuh"
+#include "launch.h"
+
+namespace eattn {
+namespace {
+
+constexpr int BM = 128;           // query rows per tile
+constexpr int BN = 64;            // keys per block (= mask block)
+constexpr int NVS = 2;            // V ring stages
+constexpr int kThreads = 192;
+constexpr uint32_t kHistBytes = 256u * BM * 4u;  // 128 KB, reused for V / P / U after the dense sweep
+
+template <int D>
+struct Cfg {
+    static constexpr int NKS = (D == 64) ? 4 : 3;          // K ring stages
+    static constexpr uint32_t kQBytes = BM * D * 2;        // 16 / 32 KB
+    static constexpr uint32_t kKBytes = BN * D * 2;        // 8 / 16 KB per stage
+    static constexpr uint32_t kPBytes = BM * BN * 2;       // 16 KB
+    static constexpr uint32_t offQ = 0;
+    static constexpr uint32_t offK = offQ + kQBytes;
+    static constexpr uint32_t offU = offK + NKS * kKBytes;  // union region
+    static constexpr uint32_t offV = offU;                  // V ring inside the union
+    static constexpr uint32_t offP = offV + NVS * kKBytes;  // P buffers [2]
+    static constexpr uint32_t offUU = offP + 2 * kPBytes;   // U buffers [2]
+    static constexpr uint32_t offSmall = offU + kHistBytes;
+    static_assert(offUU + 2 * kPBytes <= offSmall, "union region too small");
+    static constexpr uint32_t tmemCols = 512;
+    static constexpr uint32_t colO = 128;
+    static constexpr uint32_t colOb = 128 + D;
+};
+
+struct Small {
+    uint64_t q_full;
+    uint64_t k_full[4], k_empty[4];
+    uint64_t v_full[NVS], v_empty[NVS];
+    uint64_t s_full[2], s_empty[2];
+    uint64_t p_full[2], p_empty[2];
+    uint64_t o_full;
+    uint64_t ctrl;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+    int pad_;
+    int plan_kind[2];
+    TileStats st;
+    float T[260];
+    // followed by: plan_bits[2][W], next[W], mrow[2][W]
+};
+
+// OR of `pred` over the 128 compute threads (named barrier 1); every compute thread gets the result.
+__device__ __forceinline__ bool bar_or_compute(bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, 1, 128, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(out)
+        : "r"((uint32_t)pred)
+        : "memory");
+    return out != 0;
+}
+
+__device__ __forceinline__ bool block_full(int J, int n, int causal, int row0) {
+    const int last = J * BN + BN - 1;
+    return last < n && (!causal || last <= row0);
+}
+
+template <int D, int KIND>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+    using C = Cfg<D>;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    // 1024-byte alignment for the 128B-swizzled tiles
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                           ~(uintptr_t)1023);
+    Small& sm = *reinterpret_cast<Small*>(smem + C::offSmall);
+    const int W = a.nw;
+    uint32_t* plan_bits = reinterpret_cast<uint32_t*>(&sm + 1);  // [2][W]
+    uint32_t* next = plan_bits + 2 * W;                          // [W]
+    uint32_t* mrow = next + W;                                   // [2][W]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + C::offU);
+
+    const SolveParams sp = a.sp;
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int qt = a.ntiles - 1 - (int)blockIdx.x;
+    const int bh = blockIdx.y;
+    const int row0 = qt * BM;
+    const int kend = a.causal ? min(a.n, row0 + BM) : a.n;
+    const int nblk = (kend + BN - 1) / BN;
+    volatile int* abort_flag = &sm.abort_flag;
+
+    if (tid == 0) {
+        mbar_init(&sm.q_full, 1);
+        for (int i = 0; i < C::NKS; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
+        for (int i = 0; i < NVS; ++i) { mbar_init(&sm.v_full[i], 1); mbar_init(&sm.v_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.s_full[i], 1); mbar_init(&sm.s_empty[i], BM);
+            mbar_init(&sm.p_full[i], BM); mbar_init(&sm.p_empty[i], 1);
+        }
+        mbar_init(&sm.o_full, 1);
+        mbar_init(&sm.ctrl, BM);
+        mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        sm.st = TileStats{};
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, C::tmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t sQ = smem_u32(smem + C::offQ);
+    const uint32_t sK0 = smem_u32(smem + C::offK);
+    const uint32_t sV0 = smem_u32(smem + C::offV);
+    const uint32_t sP0 = smem_u32(smem + C::offP);
+    const uint32_t sU0 = smem_u32(smem + C::offUU);
+
+    if (warp == 5) {
+        // ------------------------------------------------------------------ TMA issue
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(&sm.q_full, C::kQBytes);
+            for (int c = 0; c < D / 64; ++c)
+                tma_load_3d(smem + C::offQ + c * (BM * 128), &tmQ, &sm.q_full, 64 * c, row0, bh);
+            uint32_t lc = 0, vc = 0;
+            bool ok = true;
+            for (int sw = 0; ok; ++sw) {
+                if (!(ok = wait_bounded(&sm.ctrl, sw & 1, abort_flag, a.status))) break;
+                const int kind = sm.plan_kind[sw & 1];
+                if (kind == kSweepDone) break;
+                const uint32_t* bits_p = plan_bits + (sw & 1) * W;
+                for (int wd = 0; wd < W && ok; ++wd) {
+                    uint32_t bits = bits_p[wd];
+                    while (bits && ok) {
+                        const int J = wd * 32 + __ffs(bits) - 1;
+                        bits &= bits - 1;
+                        const uint32_t ks = lc % C::NKS;
+                        if (!(ok = wait_bounded(&sm.k_empty[ks], ((lc / C::NKS) & 1) ^ 1, abort_flag, a.status))) break;
+                        mbar_arrive_expect_tx(&sm.k_full[ks], C::kKBytes);
+                        for (int c = 0; c < D / 64; ++c)
+                            tma_load_3d(smem + C::offK + ks * C::kKBytes + c * (BN * 128), &tmK, &sm.k_full[ks],
+                                        64 * c, J * BN, bh);
+                        ++lc;
+                        if (kind == kSweepPV) {
+                            const uint32_t vs = vc % NVS;
+                            if (!(ok = wait_bounded(&sm.v_empty[vs], ((vc / NVS) & 1) ^ 1, abort_flag, a.status))) break;
+                            mbar_arrive_expect_tx(&sm.v_full[vs], C::kKBytes);
+                            for (int c = 0; c < D / 64; ++c)
+                                tma_load_3d(smem + C::offV + vs * C::kKBytes + c * (BN * 128), &tmV,
+                                            &sm.v_full[vs], 64 * c, J * BN, bh);
+                            ++vc;
+                        }
+                    }
+                }
+            }
+            if (!ok) {
+                // drain copies still in flight before the CTA's shared memory is released
+                for (uint32_t i = (lc > (uint32_t)C::NKS ? lc - C::NKS : 0); i < lc; ++i)
+                    wait_drain(&sm.k_full[i % C::NKS], (i / C::NKS) & 1, 100000000ull);
+                for (uint32_t i = (vc > (uint32_t)NVS ? vc - NVS : 0); i < vc; ++i)
+                    wait_drain(&sm.v_full[i % NVS], (i / NVS) & 1, 100000000ull);
+                wait_drain(&sm.q_full, 0, 100000000ull);
+            }
+        }
+    } else if (warp == 4) {
+        // ------------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
+            constexpr uint32_t idPV = idesc_bf16_f32(BM, D, false, true);
+            uint32_t lc = 0, vc = 0, sc = 0, pc = 0;
+            bool ok = wait_bounded(&sm.q_full, 0, abort_flag, a.status);
+            tc_fence_after();
+            auto issue_S = [&](uint32_t ks) -> bool {
+                const uint32_t sb = sc & 1;
+                if (!wait_bounded(&sm.k_full[ks], (lc / C::NKS) & 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&sm.s_empty[sb], ((sc >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
+                tc_fence_after();
+                const uint32_t kbase = sK0 + ks * C::kKBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t sub = kk >> 2, off = (kk & 3) * 32;
+                    const uint64_t da = sdesc_sw128(sQ + sub * (BM * 128) + off, 16, 1024);
+                    const uint64_t db = sdesc_sw128(kbase + sub * (BN * 128) + off, 16, 1024);
+                    mma_bf16_ss(tmem + sb * BN, da, db, idS, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&sm.s_full[sb]);
+                mma_commit(&sm.k_empty[ks]);
+                ++lc;
+                ++sc;
+                return true;
+            };
+            auto issue_PV = [&](bool first) -> bool {
+                const uint32_t pb = pc & 1;
+                const uint32_t vs = vc % NVS;
+                if (!wait_bounded(&sm.p_full[pb], (pc >> 1) & 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&sm.v_full[vs], (vc / NVS) & 1, abort_flag, a.status)) return false;
+                tc_fence_after();
+                const uint32_t vbase = sV0 + vs * C::kKBytes;
+#pragma unroll
+                for (int kk = 0; kk < BN / 16; ++kk) {
+                    const uint64_t dv = sdesc_sw128(vbase + kk * 2048, BN * 128, 1024);
+                    const uint64_t dp = sdesc_sw128(sP0 + pb * C::kPBytes + kk * 32, 16, 1024);
+                    const uint64_t du = sdesc_sw128(sU0 + pb * C::kPBytes + kk * 32, 16, 1024);
+                    const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+                    mma_bf16_ss(tmem + C::colO, dp, dv, idPV, acc);
+                    mma_bf16_ss(tmem + C::colOb, du, dv, idPV, acc);
+                }
+                mma_commit(&sm.p_empty[pb]);
+                mma_commit(&sm.v_empty[vs]);
+                ++pc;
+                ++vc;
+                return true;
+            };
+            for (int sw = 0; ok; ++sw) {
+                if (!(ok = wait_bounded(&sm.ctrl, sw & 1, abort_flag, a.status))) break;
+                const int kind = sm.plan_kind[sw & 1];
+                if (kind == kSweepDone) break;
+                const uint32_t* bits_p = plan_bits + (sw & 1) * W;
+                bool pending = false, first = true;
+                for (int wd = 0; wd < W && ok; ++wd) {
+                    uint32_t bits = bits_p[wd];
+                    while (bits && ok) {
+                        bits &= bits - 1;
+                        if (!(ok = issue_S(lc % C::NKS))) break;
+                        if (kind == kSweepPV) {
+                            if (pending) {
+                                if (!(ok = issue_PV(first))) break;
+                                first = false;
+                            }
+                            pending = true;
+                        }
+                    }
+                }
+                if (ok && kind == kSweepPV) {
+                    if (pending) ok = issue_PV(first);
+                    if (ok) mma_commit(&sm.o_full);
+                }
+            }
+            // make sure every MMA has finished before TMEM is released
+            mma_commit(&sm.drain);
+            wait_drain(&sm.drain, 0, 200000000ull);
+        }
+    } else {
+        // ------------------------------------------------------------------ compute warps
+        const int r = tid;  // row within the tile == TMEM lane
+        const int row = row0 + r;
+        const bool valid = row < a.n;
+        const int n_i = valid ? allowed_keys(row, a.n, a.causal) : 1;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const size_t head = (size_t)bh * a.n;
+        const int half = r >> 6;  // which 64-row mask block of the tile
+
+        if (sp.init_mode == 0)
+            for (int s = 0; s < sp.bins; ++s) hist[s * BM + r] = 0u;
+        for (int i = r; i <= sp.bins; i += BM) sm.T[i] = (KIND == kGeneric) ? powf((float)i, sp.k) : 0.0f;
+        for (int i = r; i < W; i += BM) {
+            const int lo = i * 32;
+            uint32_t v = 0u;
+            if (lo < nblk) v = (nblk - lo >= 32) ? 0xffffffffu : ((1u << (nblk - lo)) - 1u);
+            plan_bits[i] = v;  // plan 0: every causal block
+            next[i] = 0u;
+        }
+        if (r == 0) sm.plan_kind[0] = kSweepDense;
+        named_bar_sync(1, BM);
+        mbar_arrive(&sm.ctrl);
+
+        uint32_t sc = 0, pc = 0;
+        int sw = 0;
+        bool ok = true;
+        float vbuf[BN];
+
+        // Load this row's S tile of the next block of the current sweep into vbuf (raw q.k).
+        auto load_S = [&]() -> bool {
+            const uint32_t sb = sc & 1;
+            const bool got = wait_bounded(&sm.s_full[sb], (sc >> 1) & 1, abort_flag, a.status);
+            if (!__all_sync(0xffffffffu, got)) return false;
+            tc_fence_after();
+            __syncwarp();
+            uint32_t* rr = reinterpret_cast<uint32_t*>(vbuf);
+            tmem_ld32(lane_base + sb * BN, rr);
+            tmem_ld32(lane_base + sb * BN + 32, rr + 32);
+            tmem_ld_wait();
+            tc_fence_before();
+            mbar_arrive(&sm.s_empty[sb]);
+            ++sc;
+            return true;
+        };
+        auto mask_S = [&](int J) {
+            if (block_full(J, a.n, a.causal, row0) && valid) return;
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+                const int key = J * BN + c;
+                if (!(valid && key < a.n && (!a.causal || key <= row))) vbuf[c] = -INFINITY;
+            }
+        };
+        auto publish = [&](int kind) {
+            // next[] holds the keep bits of the sweep just finished
+            named_bar_sync(1, BM);
+            const int nb = (sw + 1) & 1;
+            for (int i = r; i < W; i += BM) {
+                plan_bits[nb * W + i] = next[i];
+                next[i] = 0u;
+            }
+            if (kind == kSweepPV)
+                for (int i = r; i < 2 * W; i += BM) mrow[i] = 0u;
+            if (r == 0) sm.plan_kind[nb] = kind;
+            named_bar_sync(1, BM);
+            ++sw;
+            mbar_arrive(&sm.ctrl);
+        };
+
+        // ---- sweep 0: dense ----
+        HistRow h;
+        h.m_raw = -INFINITY;
+        h.thr_raw = INFINITY;
+        h.top = 0;
+        h.any = false;
+        for (int J = 0; J < nblk && ok; ++J) {
+            if (!(ok = load_S())) break;
+            mask_S(J);
+            float amax = vbuf[0];
+#pragma unroll
+            for (int c = 1; c < BN; ++c) amax = fmaxf(amax, vbuf[c]);
+            bool any = false;
+            if (sp.init_mode == 0) {
+                hist_raise(h, amax, sp, hist, r);
+#pragma unroll
+                for (int c = 0; c < BN; ++c)
+                    if (vbuf[c] > h.thr_raw) {
+                        any = true;
+                        hist_add(h, vbuf[c], sp, hist, r);
+                    }
+            } else {
+                if (amax > h.m_raw) { h.m_raw = amax; h.thr_raw = amax - sp.inv_cz; h.any = true; }
+#pragma unroll
+                for (int c = 0; c < BN; ++c) any |= vbuf[c] > h.thr_raw;
+            }
+            const uint32_t ball = __ballot_sync(0xffffffffu, any);
+            if (lane == 0 && ball) atomicOr(&next[J >> 5], 1u << (J & 31));
+        }
+
+        ok = !bar_or_compute(!ok || *abort_flag != 0);
+        const float m = sp.cz * h.m_raw;
+        float tau_h = m - 1.0f;
+        if (ok && valid && sp.init_mode == 0) tau_h = hist_tau<KIND>(h, sp, hist, r, sm.T);
+        RowSolve s;
+        solve_init(s, valid ? tau_h : 0.0f, valid ? m : 1.0f, n_i, sp);
+        if (!valid) s.done = true;
+        if (valid && a.tau_hist) a.tau_hist[head + row] = tau_h;
+
+        // ---- refinement sweeps ----
+        float last_step = INFINITY;
+        int refine = 0;
+        while (ok) {
+            const bool need = !s.done && (refine == 0 || fabsf(last_step) > sp.w);
+            ok = !bar_or_compute(!ok || *abort_flag != 0);
+            if (!ok) break;
+            const bool any_need = bar_or_compute(need) && refine < kMaxSteps;
+            if (!any_need) break;
+            publish(kSweepRefine);
+            float F0 = 0.f, F1 = 0.f, F2 = 0.f, F0b = 0.f;
+            const float t = s.tau, t2 = s.tau2, lo0 = s.lo;
+            const bool two = s.need_two;
+            const uint32_t* bits_p = plan_bits + (sw & 1) * W;
+            for (int wd = 0; wd < W && ok; ++wd) {
+                uint32_t bits = bits_p[wd];
+                while (bits) {
+                    const int J = wd * 32 + __ffs(bits) - 1;
+                    bits &= bits - 1;
+                    if (!(ok = load_S())) break;
+                    mask_S(J);
+                    bool keep = false;
+#pragma unroll
+                    for (int c = 0; c < BN; ++c) {
+                        const float z = sp.cz * vbuf[c];
+                        keep |= z > lo0;
+                        const float x = z - t;
+                        if (x > 0.f) add_sums<KIND>(x, sp.k, F0, F1, F2);
+                        if (two) {
+                            const float x2 = z - t2;
+                            if (x2 > 0.f) F0b += pow_k<KIND>(x2, sp.k);
+                        }
+                    }
+                    const uint32_t ball = __ballot_sync(0xffffffffu, keep);
+                    if (lane == 0 && ball) atomicOr(&next[J >> 5], 1u << (J & 31));
+                }
+            }
+            const float before = s.tau;
+            solve_step(s, F0, F1, F2, F0b, sp);
+            last_step = s.tau - before;
+            ++refine;
+        }
+
+        // ---- P V sweeps ----
+        float Su = 0.f;
+        int pv = 0;
+        while (ok) {
+            publish(kSweepPV);
+            float Sp = 0.f, F2 = 0.f;
+            Su = 0.f;
+            const float t = s.tau, lo0 = s.lo;
+            const uint32_t* bits_p = plan_bits + (sw & 1) * W;
+            for (int wd = 0; wd < W && ok; ++wd) {
+                uint32_t bits = bits_p[wd];
+                while (bits) {
+                    const int J = wd * 32 + __ffs(bits) - 1;
+                    bits &= bits - 1;
+                    if (!(ok = load_S())) break;
+                    mask_S(J);
+                    bool keep = false, nz = false;
+                    uint32_t pp[BN / 2], uu[BN / 2];
+#pragma unroll
+                    for (int c = 0; c < BN; c += 2) {
+                        float pv2[2], uv2[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const float z = sp.cz * vbuf[c + e];
+                            keep |= z > lo0;
+                            const float x = z - t;
+                            float p = 0.f, u = 0.f;
+                            if (x > 0.f) {
+                                if constexpr (KIND == kAlpha15) { u = x; p = x * x; F2 += 1.f; }
+                                else if constexpr (KIND == kAlpha2) { u = 1.f; p = x; }
+                                else { u = exp2f((sp.k - 1.f) * __log2f(x)); p = u * x; F2 += __fdividef(u, x); }
+                                nz = true;
+                            }
+                            Sp += p;
+                            Su += u;
+                            pv2[e] = p;
+                            uv2[e] = u;
+                        }
+                        pp[c / 2] = pack_bf16x2(pv2[0], pv2[1]);
+                        uu[c / 2] = pack_bf16x2(uv2[0], uv2[1]);
+                    }
+                    const uint32_t pb = pc & 1;
+                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_empty[pb], ((pc >> 1) & 1) ^ 1, abort_flag, a.status));
+                    if (!ok) break;
+                    const uint32_t pbase = sP0 + pb * Cfg<D>::kPBytes;
+                    const uint32_t ubase = sU0 + pb * Cfg<D>::kPBytes;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)ch);
+                        st_shared_v4(pbase + off, pp[4 * ch], pp[4 * ch + 1], pp[4 * ch + 2], pp[4 * ch + 3]);
+                        st_shared_v4(ubase + off, uu[4 * ch], uu[4 * ch + 1], uu[4 * ch + 2], uu[4 * ch + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(&sm.p_full[pb]);
+                    ++pc;
+                    const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+                    const uint32_t nb = __ballot_sync(0xffffffffu, nz);
+                    if (lane == 0) {
+                        if (kb) atomicOr(&next[J >> 5], 1u << (J & 31));
+                        if (nb) atomicOr(&mrow[half * W + (J >> 5)], 1u << (J & 31));
+                    }
+                }
+            }
+            ++pv;
+            const float before = s.tau;
+            solve_step(s, Sp, Su, F2, 0.f, sp);
+            const bool changed = s.tau != before;
+            ok = !bar_or_compute(!ok || *abort_flag != 0);
+            if (!ok) break;
+            if (!bar_or_compute(changed) || pv >= kMaxSteps) break;
+        }
+
+        // ---- wait for the last P V MMAs, then write O, U V, tau, sum u, mask ----
+        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(&sm.o_full, (pv - 1) & 1, abort_flag, a.status));
+        ok = !bar_or_compute(!ok || *abort_flag != 0);
+        if (ok) {
+            tc_fence_after();
+            __syncwarp();
+            __nv_bfloat16* Oh = static_cast<__nv_bfloat16*>(a.O) + head * D;
+            float* Obh = a.obar + head * D;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32], ob[32];
+                tmem_ld32(lane_base + C::colO + c0, o);
+                tmem_ld32(lane_base + C::colOb + c0, ob);
+                tmem_ld_wait();
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(Oh + (size_t)row * D + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float* f = reinterpret_cast<const float*>(o + 8 * i);
+                        dst[i] = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]),
+                                            pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
+                    }
+                    float4* dob = reinterpret_cast<float4*>(Obh + (size_t)row * D + c0);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float* f = reinterpret_cast<const float*>(ob + 4 * i);
+                        dob[i] = make_float4(f[0], f[1], f[2], f[3]);
+                    }
+                }
+            }
+            tc_fence_before();
+            if (valid) {
+                a.tau[head + row] = s.tau;
+                a.sum_u[head + row] = Su;
+                if (a.steps) a.steps[head + row] = (uint8_t)s.steps;
+            }
+        }
+        // tell the issuing warps to stop
+        if (r == 0) sm.plan_kind[(sw + 1) & 1] = kSweepDone;
+        named_bar_sync(1, BM);
+        mbar_arrive(&sm.ctrl);
+
+        // mask rows of this tile (two 64-row query blocks)
+        named_bar_sync(1, BM);
+        for (int i = r; i < 2 * W; i += BM) {
+            const int qb = qt * 2 + i / W;
+            if (qb < a.nqb) a.mask[((size_t)bh * a.nqb + qb) * W + (i % W)] = ok ? mrow[i] : 0u;
+        }
+        if (a.stats && ok) {
+            const uint32_t* cb = plan_bits + (sw & 1) * W;
+            uint32_t nzb = 0, cnd = 0;
+            for (int i = r; i < 2 * W; i += BM) nzb += __popc(mrow[i]);
+            for (int i = r; i < W; i += BM) cnd += __popc(cb[i]);
+            if (nzb) atomicAdd(&sm.st.nonzero_blocks, nzb);
+            if (cnd) atomicAdd(&sm.st.candidate_blocks, cnd);
+            if (valid) {
+                atomicAdd(&sm.st.rows, 1u);
+                atomicAdd(&sm.st.steps, (uint32_t)s.steps);
+                atomicAdd(&sm.st.fallbacks, (uint32_t)s.fallbacks);
+                atomicAdd(&sm.st.step_hist[min(s.steps, kMaxSteps)], 1u);
+            }
+            named_bar_sync(1, BM);
+            if (r == 0) {
+                sm.st.sweeps = (uint32_t)(1 + refine + pv);
+                flush_stats(a.stats, sm.st);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::tmemCols);
+    }
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------------
+namespace {
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled get_encode() {
+    static EncodeTiled fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    }
+    return fn;
+}
+
+}  // namespace
+
+// [BH, n, d] bf16 tensor, boxes of `rows` x 64 columns, 128B swizzle; zero fill past n.
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d, int rows) {
+    EncodeTiled enc = get_encode();
+    if (!enc) return cudaErrorNotSupported;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)BH};
+    cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int D, int KIND>
+static cudaError_t launch_fwd_tc_t(const FwdArgs& a, cudaStream_t stream) {
+    using C = Cfg<D>;
+    CUtensorMap tq, tk, tv;
+    cudaError_t e;
+    if ((e = make_tmap_bf16(&tq, a.Q, a.B * a.H, a.n, D, BM)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&tk, a.K, a.B * a.H, a.n, D, BN)) != cudaSuccess) return e;
+    if ((e = make_tmap_bf16(&tv, a.V, a.B * a.H, a.n, D, BN)) != cudaSuccess) return e;
+    const size_t bytes = 1024 + C::offSmall + sizeof(Small) + (size_t)5 * a.nw * 4;
+    if (bytes > 232448) return cudaErrorInvalidConfiguration;
+    auto kern = fwd_tc_kernel<D, KIND>;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
+        return e;
+    dim3 grid(a.ntiles, a.B * a.H);
+    kern<<<grid, kThreads, bytes, stream>>>(tq, tk, tv, a);
+    return cudaGetLastError();
+}
+
+size_t fwd_tc_smem_bytes(int d, int nw) {
+    const size_t small = sizeof(Small) + (size_t)5 * nw * 4;
+    return 1024 + (d == 64 ? Cfg<64>::offSmall : Cfg<128>::offSmall) + small;
+}
+
+cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream) {
+    if (a.d == 64) {
+        if (a.sp.alpha == 1.5f) return launch_fwd_tc_t<64, kAlpha15>(a, stream);
+        if (a.sp.alpha == 2.0f) return launch_fwd_tc_t<64, kAlpha2>(a, stream);
+        return launch_fwd_tc_t<64, kGeneric>(a, stream);
+    }
+    if (a.sp.alpha == 1.5f) return launch_fwd_tc_t<128, kAlpha15>(a, stream);
+    if (a.sp.alpha == 2.0f) return launch_fwd_tc_t<128, kAlpha2>(a, stream);
+    return launch_fwd_tc_t<128, kGeneric>(a, stream);
+}
+
+}  // namespace eattn

@@ -1,0 +1,62 @@
+// launch.h - host launchers implemented by the kernel files (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fwd_common.cuh"
+
+namespace eattn {
+
+cudaError_t launch_fwd_simt(const FwdArgs& a, bool fp32, cudaStream_t stream);
+cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
+size_t fwd_tc_smem_bytes(int d, int nw);
+size_t fwd_simt_smem_bytes(int d, int nkb, int mb, int nw);
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d, int rows);
+
+// maskT[bh][J][I / 32] bit I % 32 = mask[bh][I][J / 32] bit J % 32
+cudaError_t launch_mask_transpose(const uint32_t* mask, uint32_t* maskT, int BH, int nqb, int nkb, int nw, int nwq,
+                                  cudaStream_t stream);
+
+struct BwdArgs {
+    const void* Q;
+    const void* K;
+    const void* V;
+    const void* O;
+    const void* dO;
+    const float* rowstat;   // entmax: tau; softmax: lse (natural log)
+    const uint32_t* mask;   // [BH][nqb][nw], nullptr: dense (causal) traversal
+    const uint32_t* maskT;  // [BH][nkb][nwq], nullptr: dense
+    const float* obar;      // entmax: U V fp32 [BH][n][d]
+    const float* sum_u;     // entmax: [BH][n]
+    float* delta;           // [BH][n] written by the preprocess
+    void* dQ;
+    void* dK;
+    void* dV;
+    int* status;
+    int B, H, n, d;
+    int nqb, nkb, nw, nwq;
+    int causal;
+    int softmax;            // 1: softmax baseline, 0: entmax
+    float scale;
+    float cz;               // entmax: (alpha - 1) * scale
+    float k;                // entmax: 1 / (alpha - 1)
+    int kind;               // entmax AlphaKind
+};
+
+cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
+
+struct SoftmaxFwdArgs {
+    const void* Q;
+    const void* K;
+    const void* V;
+    void* O;
+    float* lse;
+    int* status;
+    int B, H, n, d, causal, ntiles;
+    float scale;
+};
+cudaError_t launch_softmax_fwd(const SoftmaxFwdArgs& a, cudaStream_t stream);
+
+}  // namespace eattn

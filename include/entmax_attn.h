@@ -1,0 +1,133 @@
+/*
+ * entmax_attn.h - C ABI of libentmax_attn.so: alpha-entmax attention on NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (AdaSplash-2, "Faster Differentiable Sparse Attention"):
+ *
+ *   s_ij = scale * q_i . k_j,  z_ij = (alpha - 1) s_ij          (j <= i when causal)
+ *   p_ij = [z_ij - tau_i]_+^(1/(alpha-1)),  with tau_i such that sum_j p_ij = 1
+ *   O_i  = sum_j p_ij v_j
+ *
+ * alpha-entmax replaces the softmax normaliser and yields exact zeros, at the cost of a root search
+ * for tau (gist.science (de) summary, section 1 "Problemstellung"; euno.news summary, "方法论" item 1).
+ * The forward builds an on-chip score histogram per query row whose left-edge root tau_h is a lower
+ * bound on tau (gist.science (de), section 2, "Streaming & Histogramm-Erstellung", "Theoretische
+ * Garantie"), refines it with a safeguarded Halley / Newton / secant solver with bisection fallback
+ * ("Hybrid Solver & Sparsity-Awareness"), records the nonzero (query block, key block) pairs in a
+ * bit-packed mask, 32 key blocks per uint32 ("Bit-Packed Block Mask"), and computes P V only on those
+ * blocks. The backward walks the same mask ("GPU-Optimierung": find-next-set and popcount over the
+ * nonzero blocks) with the entmax Jacobian dS = u (g - delta), u = p^(2 - alpha) on the support,
+ * g = dO V^T, delta = sum(u g) / sum(u).
+ *
+ * Conventions for every entry point
+ *   - Tensors are [B, H, n, d] row-major, d fastest, on the current CUDA device. bf16 tensors use
+ *     the IEEE bfloat16 bit layout. Base addresses must be 16-byte aligned (TMA), else
+ *     ENTMAX_ERR_ALIGN.
+ *   - tau, lse, and per-row statistics are float32 [B, H, n].
+ *   - block_mask is uint32 [B, H, nqb, nw] with nqb = ceil(n / mb), nkb = ceil(n / mb),
+ *     nw = ceil(nkb / 32); bit (J % 32) of word J / 32 in row I is set when some entry of query
+ *     block I and key block J is nonzero. mb is the mask block (opts->mask_block).
+ *   - All device buffers are owned by the caller. The library allocates and frees nothing, and does
+ *     not synchronise: calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL is
+ *     the legacy default stream).
+ *   - Argument errors return before any launch, with no effect. A device-side wait that runs out
+ *     (a pipeline barrier that does not complete within about two seconds) makes the kernel record
+ *     ENTMAX_ERR_TIMEOUT in a device status word and return early; entmax_attn_check() reports it.
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef ENTMAX_ATTN_H
+#define ENTMAX_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ENTMAX_OK = 0,
+    ENTMAX_ERR_INVALID = 1,     /* null pointer, bad size, alpha <= 1, workspace too small for ... */
+    ENTMAX_ERR_UNSUPPORTED = 2, /* valid but not built: d not in {64, 128}, fp32 backward, ...     */
+    ENTMAX_ERR_ALIGN = 3,       /* a tensor base address is not 16-byte aligned                    */
+    ENTMAX_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed                             */
+    ENTMAX_ERR_TIMEOUT = 5,     /* a device-side bounded wait ran out (reported by check())        */
+    ENTMAX_ERR_WORKSPACE = 6    /* workspace missing or smaller than entmax_attn_workspace_size()  */
+} entmax_status;
+
+typedef enum {
+    ENTMAX_BF16 = 0, /* bf16 inputs and outputs, fp32 accumulation on the tensor cores (tcgen05) */
+    ENTMAX_FP32 = 1  /* fp32 inputs and outputs, fp32 FMA arithmetic throughout (forward only)    */
+} entmax_dtype;
+
+/* Device-side counters, accumulated with atomics when opts->stats is non-NULL (zero it first). */
+typedef struct {
+    unsigned long long rows;             /* query rows solved                                     */
+    unsigned long long steps;            /* solver updates of tau after the histogram estimate    */
+    unsigned long long fallbacks;        /* updates that were bisection (step left the bracket)   */
+    unsigned long long step_hist[9];     /* rows by number of steps, 0..8                         */
+    unsigned long long causal_blocks;    /* (query block, key block) pairs with an allowed entry  */
+    unsigned long long candidate_blocks; /* pairs the sparse sweeps visited (128-row tiles x 64)  */
+    unsigned long long nonzero_blocks;   /* mask bits set                                         */
+    unsigned long long sweeps;           /* key sweeps over all tiles (dense + refine + P V)      */
+} entmax_stats;
+
+typedef struct {
+    float scale;            /* score scale; 0 means 1/sqrt(d)                                      */
+    int mask_block;         /* mask block mb (query and key); 0 means 64. bf16: 64; fp32: 32 or 64 */
+    int hist_bins;          /* histogram bins B; 0 means 256. Supported: 64, 128, 256              */
+    int init_mode;          /* 0: histogram start (default); 1: plain bracket start, no histogram  */
+    void* workspace;        /* device scratch, >= entmax_attn_workspace_size() bytes, 256-aligned, */
+    size_t workspace_bytes; /* kept by the caller from the forward to the matching backward        */
+    entmax_stats* stats;    /* optional device counters, may be NULL                               */
+    float* tau_hist;        /* optional device [B,H,n]: the histogram bound tau_h of each row      */
+    uint8_t* steps;         /* optional device [B,H,n]: solver steps taken by each row             */
+} entmax_opts;
+
+/* Bytes of workspace that entmax_attn_fwd/bwd (or softmax_attn_fwd/bwd) need for these sizes.
+ * Returns 0 for invalid sizes. opts may be NULL (defaults). */
+size_t entmax_attn_workspace_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts);
+
+/* Forward. Q, K, V: [B,H,n,d] inputs. O: [B,H,n,d] output (same dtype). tau: float32 [B,H,n]
+ * output, the normaliser in z units. block_mask: uint32 output as described above. alpha > 1.
+ * causal: 0 or 1. The workspace receives what the backward needs (sum_u, U V, the transposed mask).
+ * fp32 uses the FMA path; bf16 uses the tcgen05 path. */
+entmax_status entmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* tau,
+                              uint32_t* block_mask, int B, int H, int n, int d, float alpha, int causal,
+                              entmax_dtype dt, const entmax_opts* opts, void* stream);
+
+/* Backward (bf16 only). Inputs are the forward's inputs and outputs and dO; the workspace must be the
+ * one the forward filled. Outputs dQ, dK, dV: [B,H,n,d] bf16. Visits only the mask's nonzero blocks. */
+entmax_status entmax_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                              const float* tau, const uint32_t* block_mask, void* dQ, void* dK, void* dV,
+                              int B, int H, int n, int d, float alpha, int causal, entmax_dtype dt,
+                              const entmax_opts* opts, void* stream);
+
+/* Dense softmax flash attention in the same library, same tiling: the measurement baseline.
+ * lse: float32 [B,H,n] natural-log sum-exp of the scaled scores (output of fwd, input of bwd). */
+entmax_status softmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* lse,
+                               int B, int H, int n, int d, int causal, entmax_dtype dt,
+                               const entmax_opts* opts, void* stream);
+entmax_status softmax_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                               const float* lse, void* dQ, void* dK, void* dV, int B, int H, int n, int d,
+                               int causal, entmax_dtype dt, const entmax_opts* opts, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word of the current device:
+ * ENTMAX_ERR_TIMEOUT if a kernel's bounded wait ran out since the last check, ENTMAX_ERR_CUDA if the
+ * stream reports an error, else ENTMAX_OK. */
+entmax_status entmax_attn_check(void* stream);
+
+/* Test hook for the timeout path: launches one block that waits on a barrier nobody arrives at,
+ * with a limit of `limit_us` microseconds (1..2000000), then records ENTMAX_ERR_TIMEOUT and returns. */
+entmax_status entmax_attn_selftest_timeout(int limit_us, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* entmax_status_str(entmax_status s);
+
+/* Library ABI version: 1. */
+int entmax_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ENTMAX_ATTN_H */

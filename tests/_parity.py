@@ -1,0 +1,52 @@
+"""Helpers for GPU-vs-oracle parity tests (inputs from adaptive_sparse_flash_b200.inputs)."""
+import numpy as np
+
+# tolerances fixed by the benchmark spec for this path
+TAU_REL = 1e-3
+BF16_MAX_ABS = 2e-2
+BF16_MEAN_ABS = 2e-3
+FP32_ABS = 1e-4
+MASK_EXEMPT_P = 1e-3
+
+
+def to_torch(arrs, dtype, device="cuda"):
+    import torch
+    out = {}
+    for k, v in arrs.items():
+        t = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32))
+        out[k] = t.to(device=device, dtype=dtype).contiguous()
+    return out
+
+
+def unpack_mask(words: np.ndarray, nkb: int) -> np.ndarray:
+    """uint32 words [..., nw] -> bool [..., nkb]."""
+    w = np.asarray(words).astype(np.uint32)
+    bits = (w[..., :, None] >> np.arange(32, dtype=np.uint32)) & 1
+    return bits.reshape(w.shape[:-1] + (w.shape[-1] * 32,))[..., :nkb].astype(bool)
+
+
+def check_tau(tau_gpu, tau_ref, where=""):
+    tau_gpu = np.asarray(tau_gpu, np.float64)
+    err = np.abs(tau_gpu - tau_ref) / np.maximum(1.0, np.abs(tau_ref))
+    assert np.all(np.isfinite(tau_gpu)), where
+    assert err.max() <= TAU_REL, f"{where} tau rel err {err.max():.3e}"
+    return err.max()
+
+
+def check_close(gpu, ref, max_abs, mean_abs=None, where=""):
+    gpu = np.asarray(gpu, np.float64)
+    diff = np.abs(gpu - ref)
+    assert np.all(np.isfinite(gpu)), f"{where}: non-finite output"
+    assert diff.max() <= max_abs, f"{where}: max abs err {diff.max():.3e} > {max_abs}"
+    if mean_abs is not None:
+        assert diff.mean() <= mean_abs, f"{where}: mean abs err {diff.mean():.3e} > {mean_abs}"
+    return diff.max(), diff.mean()
+
+
+def check_mask(mask_gpu_words, bits_ref, bmax_ref, where=""):
+    """Bit-exact except blocks whose oracle max p < 1e-3."""
+    nkb = bits_ref.shape[-1]
+    g = unpack_mask(mask_gpu_words, nkb)
+    bad = (g != bits_ref) & ~(bmax_ref < MASK_EXEMPT_P)
+    assert not bad.any(), f"{where}: {int(bad.sum())} mask bits differ (of {bits_ref.size})"
+    return int((g != bits_ref).sum())

@@ -1,0 +1,149 @@
+"""GPU forward parity: the CUDA library against the float64 oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+
+from adaptive_sparse_flash_b200 import inputs
+from oracle import attention as oa
+from oracle import entmax as oe
+
+from _parity import (BF16_MAX_ABS, BF16_MEAN_ABS, FP32_ABS, check_close, check_mask, check_tau, to_torch)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from adaptive_sparse_flash_b200 import build
+    build.build()
+    return torch
+
+
+def _run(torch_cuda, arr, alpha, causal, dtype, **kw):
+    from adaptive_sparse_flash_b200 import binding as b
+    t = to_torch(arr, dtype)
+    res = b.forward(t["Q"], t["K"], t["V"], alpha, causal, with_debug=True, with_stats=True, **kw)
+    torch_cuda.cuda.synchronize()
+    assert b.entmax_attn_check() == 0
+    out = dict(O=res.O.float().cpu().numpy(), tau=res.tau.cpu().numpy(),
+               mask=res.mask.cpu().numpy().view(np.uint32), tau_h=res.tau_hist.cpu().numpy(),
+               steps=res.steps.cpu().numpy(), stats=b.stats_dict(res.stats))
+    return out
+
+
+def _check_all(g, ref, arr, alpha, causal, block, max_abs, mean_abs, where, hist=True):
+    check_tau(g["tau"], ref["tau"], where)
+    check_close(g["O"], ref["O"], max_abs, mean_abs, where + " O")
+    check_mask(g["mask"], ref["bits"], ref["bmax"], where + " mask")
+    if hist:
+        # histogram bound: tau_h <= tau*, and every true support entry lies above tau_h
+        assert np.all(g["tau_h"] <= ref["tau"] + 1e-5 * np.maximum(1, np.abs(ref["tau"]))), where
+    assert g["stats"]["rows"] == np.prod(g["tau"].shape)
+
+
+# ---- configuration 1: fp32, 1 x 1 x 256 x 64, non-causal, alpha 1.5, mask block 32 ----------------------
+
+def test_fp32_small_noncausal(torch_cuda):
+    arr = inputs.iid(1, 1, 256, 64, seed=0, dtype="fp32", with_dO=False)
+    ref = oa.forward(arr["Q"], arr["K"], arr["V"], 1.5, causal=False, block=32)
+    g = _run(torch_cuda, arr, 1.5, False, torch_cuda.float32, mask_block=32)
+    _check_all(g, ref, arr, 1.5, False, 32, FP32_ABS, None, "cfg1")
+
+
+# ---- configuration 2: bf16, 4 x 8 x 1024 x 64, causal, alpha in {1.5, 2}, beta in {1, 4, 16} ----------
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0])
+@pytest.mark.parametrize("beta", [1.0, 4.0, 16.0])
+def test_bf16_causal_sweep(torch_cuda, alpha, beta):
+    arr = inputs.iid(4, 8, 1024, 64, seed=0, beta=beta, with_dO=False)
+    ref = oa.forward(arr["Q"], arr["K"], arr["V"], alpha, causal=True, block=64)
+    g = _run(torch_cuda, arr, alpha, True, torch_cuda.bfloat16)
+    _check_all(g, ref, arr, alpha, True, 64, BF16_MAX_ABS, BF16_MEAN_ABS, f"cfg2 a={alpha} b={beta}")
+    print(f"cfg2 alpha={alpha} beta={beta} mean steps {g['steps'].mean():.3f} stats {g['stats']}")
+
+
+# ---- the fp32 FMA path on the same bf16-valued inputs (cross-check of the row logic) --------------------
+
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0, 3.0])
+def test_fp32_path_causal(torch_cuda, alpha):
+    arr = inputs.clustered(1, 2, 512, 64, centres=64, beta_q=4.0, seed=3, dtype="bf16", with_dO=False)
+    ref = oa.forward(arr["Q"], arr["K"], arr["V"], alpha, causal=True, block=64)
+    g = _run(torch_cuda, arr, alpha, True, torch_cuda.float32)
+    _check_all(g, ref, arr, alpha, True, 64, FP32_ABS * 10, None, f"fp32 path a={alpha}")
+
+
+# ---- alpha sweep on the clustered generator (every solver branch) -----------------------------------------
+
+@pytest.mark.parametrize("alpha", [1.25, 1.5, 2.0, 3.0])
+@pytest.mark.parametrize("beta", [1.0, 4.0])
+def test_bf16_alpha_sweep_small(torch_cuda, alpha, beta):
+    arr = inputs.clustered(1, 3, 640, 64, centres=64, beta_q=beta, seed=5, with_dO=False)
+    ref = oa.forward(arr["Q"], arr["K"], arr["V"], alpha, causal=True, block=64)
+    g = _run(torch_cuda, arr, alpha, True, torch_cuda.bfloat16)
+    _check_all(g, ref, arr, alpha, True, 64, BF16_MAX_ABS, BF16_MEAN_ABS, f"alpha sweep a={alpha} b={beta}")
+
+
+# ---- ragged lengths, non-causal, d = 128 ------------------------------------------------------------------
+
+@pytest.mark.parametrize("n", [1, 2, 63, 77, 130, 1000])
+@pytest.mark.parametrize("causal", [False, True])
+def test_bf16_ragged(torch_cuda, n, causal):
+    arr = inputs.iid(1, 2, n, 64, seed=n, beta=2.0, with_dO=False)
+    ref = oa.forward(arr["Q"], arr["K"], arr["V"], 1.5, causal=causal, block=64)
+    g = _run(torch_cuda, arr, 1.5, causal, torch_cuda.bfloat16)
+    _check_all(g, ref, arr, 1.5, causal, 64, BF16_MAX_ABS, BF16_MEAN_ABS, f"ragged n={n} causal={causal}")
+
+
+@pytest.mark.parametrize("alpha", [1.5, 2.0, 3.0])
+def test_bf16_d128(torch_cuda, alpha):
+    arr = inputs.iid(1, 2, 700, 128, seed=7, beta=4.0, with_dO=False)
+    ref = oa.forward(arr["Q"], arr["K"], arr["V"], alpha, causal=True, block=64)
+    g = _run(torch_cuda, arr, alpha, True, torch_cuda.bfloat16)
+    _check_all(g, ref, arr, alpha, True, 64, BF16_MAX_ABS, BF16_MEAN_ABS, f"d128 a={alpha}")
+
+
+# ---- degenerate rows --------------------------------------------------------------------------------------
+
+def test_bf16_equal_scores_uniform(torch_cuda):
+    # Q = 0: every score is 0, p is uniform over the allowed keys
+    arr = inputs.iid(1, 1, 300, 64, seed=9, with_dO=False)
+    arr["Q"] = np.zeros_like(arr["Q"])
+    g = _run(torch_cuda, arr, 1.5, True, torch_cuda.bfloat16)
+    V = arr["V"][0, 0].astype(np.float64)
+    ref_O = np.cumsum(V, axis=0) / np.arange(1, 301)[:, None]
+    check_close(g["O"][0, 0], ref_O, BF16_MAX_ABS, BF16_MEAN_ABS, "uniform")
+    n_i = np.arange(1, 301)
+    np.testing.assert_allclose(g["tau"][0, 0], 0.0 - n_i ** (1 - 1.5), rtol=0, atol=1e-3)
+
+
+def test_bf16_one_hot_rows(torch_cuda):
+    # very sharp scores: each row attends to its best key only
+    arr = inputs.iid(1, 2, 256, 64, seed=10, beta=64.0, with_dO=False)
+    ref = oa.forward(arr["Q"], arr["K"], arr["V"], 2.0, causal=True, block=64)
+    g = _run(torch_cuda, arr, 2.0, True, torch_cuda.bfloat16)
+    _check_all(g, ref, arr, 2.0, True, 64, BF16_MAX_ABS, BF16_MEAN_ABS, "one-hot")
+
+
+# ---- the plain-bracket start (no histogram) reaches the same result ---------------------------------------
+
+@pytest.mark.parametrize("alpha", [1.5, 3.0])
+def test_bf16_plain_bracket_start(torch_cuda, alpha):
+    arr = inputs.clustered(1, 2, 512, 64, centres=32, beta_q=4.0, seed=11, with_dO=False)
+    ref = oa.forward(arr["Q"], arr["K"], arr["V"], alpha, causal=True, block=64)
+    g = _run(torch_cuda, arr, alpha, True, torch_cuda.bfloat16, init_mode=1)
+    _check_all(g, ref, arr, alpha, True, 64, BF16_MAX_ABS, BF16_MEAN_ABS, "plain start", hist=False)
+
+
+# ---- the solver's iteration counts agree with the oracle's hybrid solver -----------------------------------
+
+def test_step_counts_reported(torch_cuda):
+    arr = inputs.clustered(1, 2, 1024, 64, centres=64, beta_q=4.0, seed=12, with_dO=False)
+    g = _run(torch_cuda, arr, 1.5, True, torch_cuda.bfloat16)
+    z = (1.5 - 1) * oa.scores(arr["Q"][0, 0], arr["K"][0, 0], 1 / 8)
+    valid = oa.allowed(np.arange(1024), 1024, True)
+    _, steps_ref, _ = oe.hybrid_solve(z, valid, 1.5)
+    print(f"mean steps gpu {g['steps'][0, 0].mean():.3f} oracle {steps_ref.mean():.3f}")
+    assert g["steps"].max() <= 8
+    assert abs(g["steps"][0, 0].mean() - steps_ref.mean()) <= 0.5
