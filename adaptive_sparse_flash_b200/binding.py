@@ -251,9 +251,9 @@ def forward(Q, K, V, alpha, causal=True, *, scale=0.0, mask_block=0, hist_bins=0
 
 def backward(Q, K, V, fwd: EntmaxForward, dO, stream=None):
     import torch
-    dQ = torch.empty_like(Q)
-    dK = torch.empty_like(K)
-    dV = torch.empty_like(V)
+    dQ = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
+    dK = torch.empty(K.shape, dtype=torch.float32, device=K.device)
+    dV = torch.empty(V.shape, dtype=torch.float32, device=V.device)
     entmax_attn_bwd(Q, K, V, fwd.O, dO, fwd.tau, fwd.mask, dQ, dK, dV, fwd.alpha, fwd.causal, fwd.opts, stream)
     return dQ, dK, dV
 
@@ -280,7 +280,7 @@ def softmax_backward(Q, K, V, O, lse, dO, causal=True, workspace=None, stream=No
     if workspace is None:
         workspace = alloc_workspace(B, H, n, d, _dtype_code(Q), Q.device)
     opts = make_opts(workspace)
-    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    dQ, dK, dV = (torch.empty(Q.shape, dtype=torch.float32, device=Q.device) for _ in range(3))
     softmax_attn_bwd(Q, K, V, O, dO, lse, dQ, dK, dV, causal, opts, stream)
     return dQ, dK, dV
 

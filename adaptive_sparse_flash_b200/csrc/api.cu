@@ -83,16 +83,20 @@ entmax_status check_dims(int B, int H, int n, int d, entmax_dtype dt, const entm
     return ENTMAX_OK;
 }
 
+// Workspace: U V (fp32 [BH][n][d]) and sum u ([BH][n]) from the forward; delta and the row statistic
+// padded to whole 64-row blocks ([BH][ceil(n/64)*64]) for the backward; the transposed mask.
 struct Workspace {
     float* obar;
     float* sum_u;
-    float* delta;
+    float* delta_pad;
+    float* stat_pad;
     uint32_t* maskT;
     size_t bytes;
 };
 
 Workspace layout(const Dims& D, void* base) {
     const size_t rows = (size_t)D.B * D.H * D.n;
+    const size_t rows_pad = (size_t)D.B * D.H * (size_t)((D.n + 63) / 64) * 64;
     Workspace w;
     char* p = static_cast<char*>(base);
     size_t off = 0;
@@ -100,8 +104,10 @@ Workspace layout(const Dims& D, void* base) {
     off = align256(off + rows * D.d * sizeof(float));
     w.sum_u = reinterpret_cast<float*>(p + off);
     off = align256(off + rows * sizeof(float));
-    w.delta = reinterpret_cast<float*>(p + off);
-    off = align256(off + rows * sizeof(float));
+    w.delta_pad = reinterpret_cast<float*>(p + off);
+    off = align256(off + rows_pad * sizeof(float));
+    w.stat_pad = reinterpret_cast<float*>(p + off);
+    off = align256(off + rows_pad * sizeof(float));
     w.maskT = reinterpret_cast<uint32_t*>(p + off);
     off = align256(off + (size_t)D.B * D.H * D.nkb * D.nwq * sizeof(uint32_t));
     w.bytes = off;
@@ -207,20 +213,88 @@ EATTN_API entmax_status entmax_attn_selftest_timeout(int limit_us, void* stream)
 
 }  // extern "C"
 
-// ---- entry points whose kernels are added in later files (placeholders until then) ----
+
+namespace {
+
+entmax_status bwd_common(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                         const float* rowstat, const uint32_t* block_mask, void* dQ, void* dK, void* dV, int B,
+                         int H, int n, int d, float alpha, int causal, entmax_dtype dt, const entmax_opts* opts,
+                         void* stream, bool softmax) {
+    if (!Q || !K || !V || !O || !dO || !rowstat || !dQ || !dK || !dV) return ENTMAX_ERR_INVALID;
+    if (!softmax && !block_mask) return ENTMAX_ERR_INVALID;
+    if (!softmax && (!(alpha > 1.0f) || !isfinite(alpha))) return ENTMAX_ERR_INVALID;
+    if (causal != 0 && causal != 1) return ENTMAX_ERR_INVALID;
+    Dims D;
+    entmax_status st = check_dims(B, H, n, d, dt, opts, &D);
+    if (st != ENTMAX_OK) return st;
+    if (dt != ENTMAX_BF16) return ENTMAX_ERR_UNSUPPORTED;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(dQ) ||
+        !aligned16(dK) || !aligned16(dV))
+        return ENTMAX_ERR_ALIGN;
+    Workspace ws;
+    if ((st = check_workspace(D, opts, &ws)) != ENTMAX_OK) return st;
+    int* status = status_ptr();
+    if (!status) return ENTMAX_ERR_CUDA;
+    const float scale = opts->scale != 0.0f ? opts->scale : 1.0f / sqrtf((float)d);
+    BwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.Q = Q; a.K = K; a.V = V; a.O = O; a.dO = dO; a.rowstat = rowstat;
+    a.mask = softmax ? nullptr : block_mask;
+    a.maskT = softmax ? nullptr : ws.maskT;
+    a.obar = ws.obar; a.sum_u = ws.sum_u;
+    a.dQ = dQ; a.dK = dK; a.dV = dV; a.status = status;
+    a.B = B; a.H = H; a.n = n; a.d = d;
+    a.nqb = D.nqb; a.nkb = D.nkb; a.nw = D.nw; a.nwq = D.nwq;
+    a.causal = causal; a.softmax = softmax ? 1 : 0; a.scale = scale;
+    if (softmax) {
+        a.cz = scale * 1.4426950408889634f;
+        a.k = 1.0f;
+        a.kind = 0;
+    } else {
+        const SolveParams sp = make_solve_params(alpha, scale, D.bins, 0);
+        a.cz = sp.cz;
+        a.k = sp.k;
+        a.kind = alpha == 1.5f ? kAlpha15 : (alpha == 2.0f ? kAlpha2 : kGeneric);
+    }
+    return from_cuda(launch_bwd(a, ws.delta_pad, ws.stat_pad, static_cast<cudaStream_t>(stream)));
+}
+
+}  // namespace
+
 extern "C" {
-EATTN_API entmax_status entmax_attn_bwd(const void*, const void*, const void*, const void*, const void*,
-                                        const float*, const uint32_t*, void*, void*, void*, int, int, int, int,
-                                        float, int, entmax_dtype, const entmax_opts*, void*) {
-    return ENTMAX_ERR_UNSUPPORTED;
+
+EATTN_API entmax_status entmax_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                        const float* tau, const uint32_t* block_mask, void* dQ, void* dK, void* dV,
+                                        int B, int H, int n, int d, float alpha, int causal, entmax_dtype dt,
+                                        const entmax_opts* opts, void* stream) {
+    return bwd_common(Q, K, V, O, dO, tau, block_mask, dQ, dK, dV, B, H, n, d, alpha, causal, dt, opts, stream,
+                      false);
 }
-EATTN_API entmax_status softmax_attn_fwd(const void*, const void*, const void*, void*, float*, int, int, int, int,
-                                         int, entmax_dtype, const entmax_opts*, void*) {
-    return ENTMAX_ERR_UNSUPPORTED;
+
+EATTN_API entmax_status softmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* lse, int B,
+                                         int H, int n, int d, int causal, entmax_dtype dt, const entmax_opts* opts,
+                                         void* stream) {
+    if (!Q || !K || !V || !O || !lse) return ENTMAX_ERR_INVALID;
+    if (causal != 0 && causal != 1) return ENTMAX_ERR_INVALID;
+    Dims D;
+    entmax_status st = check_dims(B, H, n, d, dt, opts, &D);
+    if (st != ENTMAX_OK) return st;
+    if (dt != ENTMAX_BF16) return ENTMAX_ERR_UNSUPPORTED;
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return ENTMAX_ERR_ALIGN;
+    int* status = status_ptr();
+    if (!status) return ENTMAX_ERR_CUDA;
+    SoftmaxFwdArgs a;
+    memset(&a, 0, sizeof(a));
+    a.Q = Q; a.K = K; a.V = V; a.O = O; a.lse = lse; a.status = status;
+    a.B = B; a.H = H; a.n = n; a.d = d; a.causal = causal; a.ntiles = D.ntiles;
+    a.scale = (opts && opts->scale != 0.0f) ? opts->scale : 1.0f / sqrtf((float)d);
+    return from_cuda(launch_softmax_fwd(a, static_cast<cudaStream_t>(stream)));
 }
-EATTN_API entmax_status softmax_attn_bwd(const void*, const void*, const void*, const void*, const void*,
-                                         const float*, void*, void*, void*, int, int, int, int, int, entmax_dtype,
-                                         const entmax_opts*, void*) {
-    return ENTMAX_ERR_UNSUPPORTED;
+
+EATTN_API entmax_status softmax_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                         const float* lse, void* dQ, void* dK, void* dV, int B, int H, int n, int d,
+                                         int causal, entmax_dtype dt, const entmax_opts* opts, void* stream) {
+    return bwd_common(Q, K, V, O, dO, lse, nullptr, dQ, dK, dV, B, H, n, d, 2.0f, causal, dt, opts, stream, true);
 }
-}
+
+}  // extern "C"

@@ -25,7 +25,8 @@ namespace eattn {
 enum AlphaKind : int { kGeneric = 0, kAlpha2 = 1, kAlpha15 = 2 };
 enum Method : int { kHalley = 0, kNewton = 1, kSecant = 2 };
 
-constexpr int kMaxSteps = 8;
+constexpr int kMaxSteps = 8;  // last bin of the step histogram ("8 or more")
+constexpr int kMaxSweeps = 30;
 constexpr float kFtol = 1e-5f;
 constexpr float kXtol = 1e-6f;
 constexpr int kTileRows = 128;  // query rows per CTA; hist slot s of row r lives at hist[s * 128 + r]
@@ -79,18 +80,59 @@ __device__ __forceinline__ void add_sums(float x, float k, float& F0, float& F1,
 }
 
 // ---------------------------------------------------------------------------------------------
-// Histogram ring (thread-owned row). hist: u32 [B slots][128 rows].
+// Histogram ring (thread-owned row). hist: u32 [B slots][128 rows]. A 256-bit mask in registers
+// marks which slots hold a bin of the current window, so sliding the window clears bits instead of
+// shared memory, and the histogram needs no zeroing before use.
 // ---------------------------------------------------------------------------------------------
 struct HistRow {
     float m_raw;    // running max of the raw score
     float thr_raw;  // raw threshold for binning: z > m_run - 1
     int top;        // bin index of the running max
     bool any;       // any entry seen
+    uint32_t live[8];  // slot s holds a counted bin of the window iff bit s of live is set
 };
+
+__device__ __forceinline__ void hist_init(HistRow& h) {
+    h.m_raw = -INFINITY;
+    h.thr_raw = INFINITY;
+    h.top = 0;
+    h.any = false;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h.live[i] = 0u;
+}
 
 __device__ __forceinline__ int bin_of(float a, float cbin) {
     float y = fminf(fmaxf(a * cbin, -1.0e9f), 1.0e9f);
     return __float2int_rd(y);
+}
+
+__device__ __forceinline__ bool slot_live(const HistRow& h, int s) {
+    uint32_t w = 0u;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) w = (i == (s >> 5)) ? h.live[i] : w;
+    return (w >> (s & 31)) & 1u;
+}
+
+// Clear the live bits of the `len` slots starting at slot `s0` (circular over B slots, len < B).
+__host__ __device__ __forceinline__ void live_clear(HistRow& h, int s0, int len, int B) {
+    // bits [s0, s0 + len) of a B-bit ring; B <= 256 and a power of two
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int lo = i * 32;
+        if (lo >= B) break;
+        // positions p in [lo, lo+32) with (p - s0) mod B < len
+        uint32_t m = 0u;
+        const int a0 = ((lo - s0) % B + B) % B;  // offset of bit 0 of this word from s0
+        if (a0 < len) m = (len - a0 >= 32) ? 0xffffffffu : ((1u << (len - a0)) - 1u);
+        // the run may wrap into the top of this word
+        const int wrap = a0 + 32 - B;  // bits of this word whose offset wrapped past B
+        if (wrap > 0) {
+            const int first = 32 - wrap;  // bit index where offset wraps to 0
+            const int cnt = min(wrap, len);
+            if (cnt > 0) m |= ((cnt >= 32) ? 0xffffffffu : ((1u << cnt) - 1u)) << first;
+        }
+        h.live[i] &= ~m;
+    }
 }
 
 // Raise the running max to `a_max` (raw) and slide the window.
@@ -99,8 +141,13 @@ __device__ __forceinline__ void hist_raise(HistRow& h, float a_max, const SolveP
     const int nt = bin_of(a_max, sp.cbin);
     const int B = sp.bins;
     if (h.any && nt > h.top) {
-        const int steps = min(nt - h.top, B);
-        for (int t = 1; t <= steps; ++t) hist[((h.top + t) & (B - 1)) * kTileRows + r] = 0u;
+        const int d = nt - h.top;
+        if (d >= B) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) h.live[i] = 0u;
+        } else {
+            live_clear(h, (h.top + 1) & (B - 1), d, B);
+        }
     }
     h.top = h.any ? max(h.top, nt) : nt;
     h.any = true;
@@ -109,10 +156,21 @@ __device__ __forceinline__ void hist_raise(HistRow& h, float a_max, const SolveP
 }
 
 // Bin one raw score that passed a > thr_raw.
-__device__ __forceinline__ void hist_add(const HistRow& h, float a, const SolveParams& sp, uint32_t* hist, int r) {
+__device__ __forceinline__ void hist_add(HistRow& h, float a, const SolveParams& sp, uint32_t* hist, int r) {
     const int b = bin_of(a, sp.cbin);
     const int j = h.top - b;
-    if (j >= 0 && j < sp.bins) hist[(b & (sp.bins - 1)) * kTileRows + r] += 1u;
+    if (j >= 0 && j < sp.bins) {
+        const int s = b & (sp.bins - 1);
+        uint32_t* c = &hist[s * kTileRows + r];
+        if (slot_live(h, s)) {
+            *c += 1u;
+        } else {
+            *c = 1u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i == (s >> 5)) h.live[i] |= 1u << (s & 31);
+        }
+    }
 }
 
 // Root tau_h of the left-edge binned function, in z units (a lower bound on tau*).
@@ -123,7 +181,10 @@ template <int KIND>
 __device__ float hist_tau(const HistRow& h, const SolveParams& sp, const uint32_t* hist, int r, const float* T) {
     const int B = sp.bins;
     const float Bm1 = (float)(B - 1);
-    auto cnt = [&](int j) -> float { return (float)hist[((h.top - j) & (B - 1)) * kTileRows + r]; };
+    auto cnt = [&](int j) -> float {
+        const int sl = (h.top - j) & (B - 1);
+        return slot_live(h, sl) ? (float)hist[sl * kTileRows + r] : 0.0f;
+    };
     if constexpr (KIND == kAlpha15 || KIND == kAlpha2) {
         // A0 = sum c_j, A1 = sum c_j (J - j), A2 = sum c_j (J - j)^2 over offsets j < J (exact integers)
         double A0 = 0.0, A1 = 0.0, A2 = 0.0;
@@ -186,14 +247,24 @@ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, const uint32_
 
 // ---------------------------------------------------------------------------------------------
 // Solver state and step
+//
+// Halley / Newton: open steps from the current tau, kept inside the bracket [lo, hi] (bisection
+// otherwise); stop at |f| <= ftol, a step <= xtol max(1, |tau|), or the step cap.
+// Secant (alpha > 2): bracketing (Illinois) secant. The first sweep evaluates f at both bracket
+// ends; each step takes the secant through the current ends and the new point replaces the end of
+// the same sign, halving the f value of an end kept twice in a row. Stop at |f| <= ftol, a bracket
+// narrower than ~4 float32 ulps of tau, or the step cap.
 // ---------------------------------------------------------------------------------------------
+constexpr float kXtolBracket = 4.8e-7f;
+
 struct RowSolve {
     float tau, lo, hi;
-    float prev_t, prev_f;  // secant: the other point
-    float tau2;            // secant: second point evaluated in the first refinement sweep
-    int steps, fallbacks;
+    float flo, fhi;  // secant: f at the bracket ends
+    float tau2;      // secant: the second point evaluated in the first refinement sweep
+    int side;        // secant: which end the last point replaced (+1 lo, -1 hi)
+    int steps, fallbacks, max_steps;
     bool done;
-    bool need_two;  // secant: the next sweep also evaluates f at tau2
+    bool need_two;   // secant: the next sweep also evaluates f at tau2
 };
 
 // Initial bracket from the histogram bound (or the plain bracket), for a row with max z `m` and
@@ -210,13 +281,24 @@ __device__ __forceinline__ void solve_init(RowSolve& s, float tau_h, float m, in
     s.lo = lo;
     s.hi = hi;
     s.tau = lo;
-    s.prev_t = hi;
-    s.prev_f = 0.0f;
     s.tau2 = hi;
+    s.flo = 0.0f;
+    s.fhi = 0.0f;
+    s.side = 0;
     s.steps = 0;
     s.fallbacks = 0;
+    s.max_steps = sp.init_mode == 0 ? 12 : 24;
     s.done = false;
     s.need_two = (sp.method == kSecant);
+}
+
+__device__ __forceinline__ void secant_next(RowSolve& s) {
+    const float cand = s.hi - s.fhi * (s.hi - s.lo) / (s.fhi - s.flo);
+    const bool ok = isfinite(cand) && cand > s.lo && cand < s.hi;
+    s.tau = ok ? cand : 0.5f * (s.lo + s.hi);
+    s.fallbacks += ok ? 0 : 1;
+    s.steps += 1;
+    if (s.hi - s.lo <= kXtolBracket * fmaxf(1.0f, fabsf(s.tau)) || s.steps >= s.max_steps) s.done = true;
 }
 
 // One solver update from the sums at the current tau (F0 = sum x^k, F1 = sum x^(k-1),
@@ -224,14 +306,31 @@ __device__ __forceinline__ void solve_init(RowSolve& s, float tau_h, float m, in
 __device__ __forceinline__ void solve_step(RowSolve& s, float F0, float F1, float F2, float F0b,
                                            const SolveParams& sp) {
     if (s.done) return;
-    if (s.need_two) {
-        // secant start: (tau2, f(tau2)) is the other point; it is a bracket end if its sign says so
-        s.need_two = false;
-        const float fb = F0b - 1.0f;
-        s.prev_t = s.tau2;
-        s.prev_f = fb;
-        if (fb <= 0.0f) s.hi = fminf(s.hi, s.tau2);
-        else s.lo = fmaxf(s.lo, s.tau2);
+    if (sp.method == kSecant) {
+        if (s.need_two) {
+            s.need_two = false;
+            const float fa = F0 - 1.0f, fb = F0b - 1.0f;
+            // an end whose sign contradicts the bracket is off only by rounding: accept it
+            if (fabsf(fa) <= kFtol || fa < 0.0f) { s.done = true; return; }
+            if (fabsf(fb) <= kFtol || fb > 0.0f) { s.tau = s.tau2; s.done = true; return; }
+            s.flo = fa;
+            s.fhi = fb;
+            secant_next(s);
+            return;
+        }
+        const float fc = F0 - 1.0f;
+        if (fabsf(fc) <= kFtol) { s.done = true; return; }
+        if (fc > 0.0f) {
+            s.lo = s.tau; s.flo = fc;
+            if (s.side == 1) s.fhi *= 0.5f;
+            s.side = 1;
+        } else {
+            s.hi = s.tau; s.fhi = fc;
+            if (s.side == -1) s.flo *= 0.5f;
+            s.side = -1;
+        }
+        secant_next(s);
+        return;
     }
     const float f = F0 - 1.0f;
     if (fabsf(f) <= kFtol) { s.done = true; return; }
@@ -242,12 +341,8 @@ __device__ __forceinline__ void solve_step(RowSolve& s, float F0, float F1, floa
     if (sp.method == kHalley) {
         const float fpp = k * (k - 1.0f) * F2;
         cand = s.tau - 2.0f * f * fp / (2.0f * fp * fp - f * fpp);
-    } else if (sp.method == kNewton) {
-        cand = s.tau - f / fp;
     } else {
-        cand = s.tau - f * (s.tau - s.prev_t) / (f - s.prev_f);
-        s.prev_t = s.tau;
-        s.prev_f = f;
+        cand = s.tau - f / fp;
     }
     const bool ok = isfinite(cand) && cand > s.lo && cand < s.hi;
     const float nt = ok ? cand : 0.5f * (s.lo + s.hi);
@@ -255,7 +350,7 @@ __device__ __forceinline__ void solve_step(RowSolve& s, float F0, float F1, floa
     s.steps += 1;
     const bool small = fabsf(nt - s.tau) <= kXtol * fmaxf(1.0f, fabsf(s.tau));
     s.tau = nt;
-    if (small || s.steps >= kMaxSteps) s.done = true;
+    if (small || s.steps >= s.max_steps) s.done = true;
 }
 
 }  // namespace eattn

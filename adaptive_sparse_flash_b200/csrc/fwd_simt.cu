@@ -92,7 +92,6 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
 #pragma unroll
     for (int c = 0; c < D; ++c) q[c] = valid ? to_f<T>(Qh[(size_t)row * D + c]) : 0.0f;
 
-    for (int s = 0; s < B; ++s) hist[s * kTileRows + tid] = 0u;
     for (int i = tid; i <= B; i += blockDim.x) Tk[i] = (KIND == kGeneric) ? powf((float)i, sp.k) : 0.0f;
     for (int i = tid; i < cwords; i += blockDim.x) cand[i] = next[i] = 0u;
     if (tid == 0) {
@@ -104,10 +103,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
 
     // ---- sweep 1: dense scores, running max, histogram, candidate blocks ----
     HistRow h;
-    h.m_raw = -INFINITY;
-    h.thr_raw = INFINITY;
-    h.top = 0;
-    h.any = false;
+    hist_init(h);
     for (int J = 0; J < nblk; ++J) {
         __syncthreads();
         stage<T, D>(sK, Kh, J * mb, mb, a.n);
@@ -148,11 +144,10 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
     if (valid && a.tau_hist) a.tau_hist[head + row] = tau_h;
     int sweeps = 1;
 
-    // ---- refinement sweeps: solver sums only ----
+    // ---- refinement sweep: solver sums only ----
     float last_step = INFINITY;
-    for (int refine = 0; refine < kMaxSteps; ++refine) {
-        const bool need = !s.done && (refine == 0 || fabsf(last_step) > sp.w);
-        if (!__syncthreads_or(need)) break;
+    int refine = 0, pv = 0;
+    auto refine_sweep = [&]() {
         for (int i = tid; i < cwords; i += blockDim.x) next[i] = 0u;
         __syncthreads();
         float F0 = 0.f, F1 = 0.f, F2 = 0.f, F0b = 0.f;
@@ -185,14 +180,15 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
         const float before = s.tau;
         solve_step(s, F0, F1, F2, F0b, sp);
         last_step = s.tau - before;
+        ++refine;
         ++sweeps;
         __syncthreads();
         for (int i = tid; i < cwords; i += blockDim.x) cand[i] = next[i];
-    }
+    };
 
-    // ---- P V sweeps: O, U V, sum u, exact mask; the sums double as the check of sum p = 1 ----
+    // ---- P V sweep: O, U V, sum u, exact mask; the sums double as the check of sum p = 1 ----
     float Su = 0.f;
-    for (int pv = 0; pv < kMaxSteps; ++pv) {
+    auto pv_sweep = [&]() -> bool {
         __syncthreads();
         for (int i = tid; i < cwords; i += blockDim.x) next[i] = 0u;
         for (int i = tid; i < mrows * a.nw; i += blockDim.x) mrow[i] = 0u;
@@ -237,12 +233,24 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
             }
         }
         ++sweeps;
+        ++pv;
         const float before = s.tau;
         solve_step(s, Sp, Su, F2, 0.f, sp);
         const bool changed = s.tau != before;
         __syncthreads();
         for (int i = tid; i < cwords; i += blockDim.x) cand[i] = next[i];
-        if (!__syncthreads_or(changed)) break;
+        return __syncthreads_or(changed) != 0;
+    };
+
+    // refine while a row still takes steps wider than one bin; P V (also the check of sum p = 1);
+    // if a tau moved, refine until every row stopped and finish with one more P V sweep
+    do {
+        refine_sweep();
+    } while (refine < kMaxSweeps && __syncthreads_or(!s.done && fabsf(last_step) > sp.w));
+    while (true) {
+        const bool changed = pv_sweep();
+        if (!changed || pv >= 3) break;
+        while (refine < kMaxSweeps && __syncthreads_or(!s.done)) refine_sweep();
     }
 
     // ---- outputs ----

@@ -43,8 +43,9 @@ struct Cfg {
     static constexpr uint32_t offK = offQ + kQBytes;
     static constexpr uint32_t offU = offK + NKS * kKBytes;  // union region
     static constexpr uint32_t offV = offU;                  // V ring inside the union
-    static constexpr uint32_t offP = offV + NVS * kKBytes;  // P buffers [2]
-    static constexpr uint32_t offUU = offP + 2 * kPBytes;   // U buffers [2]
+    static constexpr uint32_t offP = offV + NVS * kKBytes;  // P buffers [2] (bf16 high part)
+    static constexpr uint32_t offPL = offP + 2 * kPBytes;   // P buffers [2] (bf16 low part)
+    static constexpr uint32_t offUU = offPL + 2 * kPBytes;  // U buffers [2]
     static constexpr uint32_t offSmall = offU + kHistBytes;
     static_assert(offUU + 2 * kPBytes <= offSmall, "union region too small");
     static constexpr uint32_t tmemCols = 512;
@@ -82,6 +83,12 @@ __device__ __forceinline__ bool bar_or_compute(bool pred) {
         : "r"((uint32_t)pred)
         : "memory");
     return out != 0;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
 }
 
 __device__ __forceinline__ bool block_full(int J, int n, int causal, int row0) {
@@ -143,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sK0 = smem_u32(smem + C::offK);
     const uint32_t sV0 = smem_u32(smem + C::offV);
     const uint32_t sP0 = smem_u32(smem + C::offP);
+    const uint32_t sPL0 = smem_u32(smem + C::offPL);
     const uint32_t sU0 = smem_u32(smem + C::offUU);
 
     if (warp == 5) {
@@ -232,9 +240,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t dv = sdesc_sw128(vbase + kk * 2048, BN * 128, 1024);
                     const uint64_t dp = sdesc_sw128(sP0 + pb * C::kPBytes + kk * 32, 16, 1024);
+                    const uint64_t dpl = sdesc_sw128(sPL0 + pb * C::kPBytes + kk * 32, 16, 1024);
                     const uint64_t du = sdesc_sw128(sU0 + pb * C::kPBytes + kk * 32, 16, 1024);
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+                    // P = P_hi + P_lo (two bf16 terms) keeps P V accurate to ~16 mantissa bits
                     mma_bf16_ss(tmem + C::colO, dp, dv, idPV, acc);
+                    mma_bf16_ss(tmem + C::colO, dpl, dv, idPV, 1u);
                     mma_bf16_ss(tmem + C::colOb, du, dv, idPV, acc);
                 }
                 mma_commit(&sm.p_empty[pb]);
@@ -282,8 +293,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const size_t head = (size_t)bh * a.n;
         const int half = r >> 6;  // which 64-row mask block of the tile
 
-        if (sp.init_mode == 0)
-            for (int s = 0; s < sp.bins; ++s) hist[s * BM + r] = 0u;
         for (int i = r; i <= sp.bins; i += BM) sm.T[i] = (KIND == kGeneric) ? powf((float)i, sp.k) : 0.0f;
         for (int i = r; i < W; i += BM) {
             const int lo = i * 32;
@@ -341,37 +350,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive(&sm.ctrl);
         };
 
+        // 8 groups of 8 scores: group maxima (3-input max), the block max, and per-group tests that
+        // skip the rare-path work for groups without a candidate entry.
+        float gm[8];
+        auto group_max = [&]() -> float {
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+                const float* v = vbuf + 8 * g;
+                gm[g] = fmax3(fmax3(v[0], v[1], v[2]), fmax3(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+            }
+            return fmax3(fmax3(gm[0], gm[1], gm[2]), fmax3(gm[3], gm[4], gm[5]), fmaxf(gm[6], gm[7]));
+        };
+
         // ---- sweep 0: dense ----
         HistRow h;
-        h.m_raw = -INFINITY;
-        h.thr_raw = INFINITY;
-        h.top = 0;
-        h.any = false;
+        hist_init(h);
         for (int J = 0; J < nblk && ok; ++J) {
             if (!(ok = load_S())) break;
             mask_S(J);
-            float amax = vbuf[0];
-#pragma unroll
-            for (int c = 1; c < BN; ++c) amax = fmaxf(amax, vbuf[c]);
+            const float amax = group_max();
             bool any = false;
             if (sp.init_mode == 0) {
                 hist_raise(h, amax, sp, hist, r);
+                if (amax > h.thr_raw) {
+                    any = true;
 #pragma unroll
-                for (int c = 0; c < BN; ++c)
-                    if (vbuf[c] > h.thr_raw) {
-                        any = true;
-                        hist_add(h, vbuf[c], sp, hist, r);
+                    for (int g = 0; g < 8; ++g) {
+                        if (gm[g] > h.thr_raw) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                if (vbuf[8 * g + e] > h.thr_raw) hist_add(h, vbuf[8 * g + e], sp, hist, r);
+                        }
                     }
+                }
             } else {
                 if (amax > h.m_raw) { h.m_raw = amax; h.thr_raw = amax - sp.inv_cz; h.any = true; }
-#pragma unroll
-                for (int c = 0; c < BN; ++c) any |= vbuf[c] > h.thr_raw;
+                any = amax > h.thr_raw;
             }
             const uint32_t ball = __ballot_sync(0xffffffffu, any);
             if (lane == 0 && ball) atomicOr(&next[J >> 5], 1u << (J & 31));
         }
-
         ok = !bar_or_compute(!ok || *abort_flag != 0);
+
         const float m = sp.cz * h.m_raw;
         float tau_h = m - 1.0f;
         if (ok && valid && sp.init_mode == 0) tau_h = hist_tau<KIND>(h, sp, hist, r, sm.T);
@@ -380,15 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!valid) s.done = true;
         if (valid && a.tau_hist) a.tau_hist[head + row] = tau_h;
 
-        // ---- refinement sweeps ----
+        // ---- refinement sweep: solver sums at the current tau over the candidate blocks ----
         float last_step = INFINITY;
-        int refine = 0;
-        while (ok) {
-            const bool need = !s.done && (refine == 0 || fabsf(last_step) > sp.w);
-            ok = !bar_or_compute(!ok || *abort_flag != 0);
-            if (!ok) break;
-            const bool any_need = bar_or_compute(need) && refine < kMaxSteps;
-            if (!any_need) break;
+        int refine = 0, pv = 0;
+        auto refine_sweep = [&]() {
             publish(kSweepRefine);
             float F0 = 0.f, F1 = 0.f, F2 = 0.f, F0b = 0.f;
             const float t = s.tau, t2 = s.tau2, lo0 = s.lo;
@@ -401,16 +416,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bits &= bits - 1;
                     if (!(ok = load_S())) break;
                     mask_S(J);
-                    bool keep = false;
+                    const float amax = group_max();
+                    const bool keep = sp.cz * amax > lo0;
+                    if (sp.cz * amax - t > 0.f) {
 #pragma unroll
-                    for (int c = 0; c < BN; ++c) {
-                        const float z = sp.cz * vbuf[c];
-                        keep |= z > lo0;
-                        const float x = z - t;
-                        if (x > 0.f) add_sums<KIND>(x, sp.k, F0, F1, F2);
-                        if (two) {
-                            const float x2 = z - t2;
-                            if (x2 > 0.f) F0b += pow_k<KIND>(x2, sp.k);
+                        for (int g = 0; g < 8; ++g) {
+                            if (sp.cz * gm[g] - t > 0.f) {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    const float z = sp.cz * vbuf[8 * g + e];
+                                    const float x = z - t;
+                                    if constexpr (KIND == kAlpha15) {
+                                        const float xp = fmaxf(x, 0.f);
+                                        F0 = fmaf(xp, xp, F0);
+                                        F1 += xp;
+                                        F2 += x > 0.f ? 1.f : 0.f;
+                                    } else if constexpr (KIND == kAlpha2) {
+                                        F0 += fmaxf(x, 0.f);
+                                        F1 += x > 0.f ? 1.f : 0.f;
+                                    } else {
+                                        if (x > 0.f) add_sums<KIND>(x, sp.k, F0, F1, F2);
+                                    }
+                                    if (two) {
+                                        const float x2 = z - t2;
+                                        if (x2 > 0.f) F0b += pow_k<KIND>(x2, sp.k);
+                                    }
+                                }
+                            }
                         }
                     }
                     const uint32_t ball = __ballot_sync(0xffffffffu, keep);
@@ -421,12 +453,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             solve_step(s, F0, F1, F2, F0b, sp);
             last_step = s.tau - before;
             ++refine;
-        }
+            ok = !bar_or_compute(!ok || *abort_flag != 0);
+        };
 
-        // ---- P V sweeps ----
+        // ---- P V sweep: p, u to shared memory for the P V / U V MMAs, exact mask, sum check ----
         float Su = 0.f;
-        int pv = 0;
-        while (ok) {
+        auto pv_sweep = [&]() -> bool {
             publish(kSweepPV);
             float Sp = 0.f, F2 = 0.f;
             Su = 0.f;
@@ -439,41 +471,58 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bits &= bits - 1;
                     if (!(ok = load_S())) break;
                     mask_S(J);
-                    bool keep = false, nz = false;
-                    uint32_t pp[BN / 2], uu[BN / 2];
-#pragma unroll
-                    for (int c = 0; c < BN; c += 2) {
-                        float pv2[2], uv2[2];
-#pragma unroll
-                        for (int e = 0; e < 2; ++e) {
-                            const float z = sp.cz * vbuf[c + e];
-                            keep |= z > lo0;
-                            const float x = z - t;
-                            float p = 0.f, u = 0.f;
-                            if (x > 0.f) {
-                                if constexpr (KIND == kAlpha15) { u = x; p = x * x; F2 += 1.f; }
-                                else if constexpr (KIND == kAlpha2) { u = 1.f; p = x; }
-                                else { u = exp2f((sp.k - 1.f) * __log2f(x)); p = u * x; F2 += __fdividef(u, x); }
-                                nz = true;
-                            }
-                            Sp += p;
-                            Su += u;
-                            pv2[e] = p;
-                            uv2[e] = u;
-                        }
-                        pp[c / 2] = pack_bf16x2(pv2[0], pv2[1]);
-                        uu[c / 2] = pack_bf16x2(uv2[0], uv2[1]);
-                    }
+                    const float amax = group_max();
+                    const bool keep = sp.cz * amax > lo0;
+                    const bool nz = sp.cz * amax - t > 0.f;
                     const uint32_t pb = pc & 1;
-                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.p_empty[pb], ((pc >> 1) & 1) ^ 1, abort_flag, a.status));
+                    ok = __all_sync(0xffffffffu,
+                                    wait_bounded(&sm.p_empty[pb], ((pc >> 1) & 1) ^ 1, abort_flag, a.status));
                     if (!ok) break;
                     const uint32_t pbase = sP0 + pb * Cfg<D>::kPBytes;
+                    const uint32_t plbase = sPL0 + pb * Cfg<D>::kPBytes;
                     const uint32_t ubase = sU0 + pb * Cfg<D>::kPBytes;
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)ch);
-                        st_shared_v4(pbase + off, pp[4 * ch], pp[4 * ch + 1], pp[4 * ch + 2], pp[4 * ch + 3]);
-                        st_shared_v4(ubase + off, uu[4 * ch], uu[4 * ch + 1], uu[4 * ch + 2], uu[4 * ch + 3]);
+                    for (int g = 0; g < 8; ++g) {
+                        uint32_t ph[4] = {0u, 0u, 0u, 0u}, pl[4] = {0u, 0u, 0u, 0u}, uu[4] = {0u, 0u, 0u, 0u};
+                        if (sp.cz * gm[g] - t > 0.f) {
+#pragma unroll
+                            for (int e = 0; e < 8; e += 2) {
+                                float pv2[2], uv2[2];
+#pragma unroll
+                                for (int q = 0; q < 2; ++q) {
+                                    const float x = sp.cz * vbuf[8 * g + e + q] - t;
+                                    float p, u;
+                                    if constexpr (KIND == kAlpha15) {
+                                        u = fmaxf(x, 0.f);
+                                        p = u * u;
+                                        F2 += x > 0.f ? 1.f : 0.f;
+                                    } else if constexpr (KIND == kAlpha2) {
+                                        p = fmaxf(x, 0.f);
+                                        u = x > 0.f ? 1.f : 0.f;
+                                    } else {
+                                        const bool pos = x > 0.f;
+                                        const float xs = pos ? x : 1.f;
+                                        const float uu1 = exp2f((sp.k - 1.f) * __log2f(xs));
+                                        u = pos ? uu1 : 0.f;
+                                        p = u * xs;
+                                        F2 += pos ? __fdividef(uu1, xs) : 0.f;
+                                    }
+                                    Sp += p;
+                                    Su += u;
+                                    pv2[q] = p;
+                                    uv2[q] = u;
+                                }
+                                const __nv_bfloat162 hi = __floats2bfloat162_rn(pv2[0], pv2[1]);
+                                const float2 hf = __bfloat1622float2(hi);
+                                ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hi);
+                                pl[e / 2] = pack_bf16x2(pv2[0] - hf.x, pv2[1] - hf.y);
+                                uu[e / 2] = pack_bf16x2(uv2[0], uv2[1]);
+                            }
+                        }
+                        const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)g);
+                        st_shared_v4(pbase + off, ph[0], ph[1], ph[2], ph[3]);
+                        st_shared_v4(plbase + off, pl[0], pl[1], pl[2], pl[3]);
+                        st_shared_v4(ubase + off, uu[0], uu[1], uu[2], uu[3]);
                     }
                     fence_proxy_async_smem();
                     mbar_arrive(&sm.p_full[pb]);
@@ -491,8 +540,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             solve_step(s, Sp, Su, F2, 0.f, sp);
             const bool changed = s.tau != before;
             ok = !bar_or_compute(!ok || *abort_flag != 0);
-            if (!ok) break;
-            if (!bar_or_compute(changed) || pv >= kMaxSteps) break;
+            return ok && bar_or_compute(changed);
+        };
+
+        // Schedule: refine while some row still takes steps wider than one bin; then P V, whose sums
+        // double as the check of sum p = 1. If any tau still moved, refine until every row has
+        // stopped (cheaper than repeated P V sweeps) and finish with one more P V sweep.
+        if (ok) {
+            do {
+                refine_sweep();
+            } while (ok && refine < kMaxSweeps &&
+                     bar_or_compute(!s.done && fabsf(last_step) > sp.w));
+        }
+        while (ok) {
+            const bool changed = pv_sweep();
+            if (!ok || !changed || pv >= 3) break;
+            while (ok && refine < kMaxSweeps && bar_or_compute(!s.done)) refine_sweep();
         }
 
         // ---- wait for the last P V MMAs, then write O, U V, tau, sum u, mask ----

@@ -30,7 +30,6 @@ struct BwdArgs {
     const uint32_t* maskT;  // [BH][nkb][nwq], nullptr: dense
     const float* obar;      // entmax: U V fp32 [BH][n][d]
     const float* sum_u;     // entmax: [BH][n]
-    float* delta;           // [BH][n] written by the preprocess
     void* dQ;
     void* dK;
     void* dV;
@@ -45,7 +44,8 @@ struct BwdArgs {
     int kind;               // entmax AlphaKind
 };
 
-cudaError_t launch_bwd(const BwdArgs& a, cudaStream_t stream);
+cudaError_t launch_bwd(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaStream_t stream);
+size_t bwd_smem_bytes(int d, int nw, int nwq);
 
 struct SoftmaxFwdArgs {
     const void* Q;

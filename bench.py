@@ -1,0 +1,362 @@
+"""Benchmark: alpha-entmax attention forward + backward on B200, effective TFLOP/s at n = 16k.
+
+One step = entmax_attn_fwd + entmax_attn_bwd over one batch of the long-context workload
+(B=1, H=16, n=16384, d=64, bf16, causal, alpha=1.5, keys clustered around 256 centres, queries
+6x their centre plus noise; V and dO ~ N(0,1)), inputs resident in HBM. Effective FLOPs count the
+dense Q K^T pass over the causal entries plus the P V and backward products of the nonzero
+64 x 64 mask blocks only:  2 d n(n+1)/2 + (2 + 5 * 2) d 64 64 N_nz  per head.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-sweep]
+
+Prints one JSON line (rank 0). Under torchrun each rank runs its own copy of the workload (independent
+heads: no data-path collective), times on its device, and the max over ranks is reported.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+B, H, N, D, ALPHA = 1, 16, 16384, 64, 1.5
+CENTRES, BETA_Q = 256, 6.0
+BLOCK = 64
+METRIC = "α-entmax attn fwd+bwd effective TFLOP/s at n=16k vs sparsity; % bf16 peak"
+WORKLOAD = (f"alpha-entmax attention fwd+bwd, B={B} H={H} n={N} d={D} bf16 causal alpha={ALPHA}, "
+            f"keys clustered on {CENTRES} centres (noise 0.3), queries {BETA_Q:g} x centre + noise")
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            j = json.load(fh)
+        return j.get("bf16_tflops", 1590.0), j.get("bf16_tflops_sustained", 1400.0), j.get("hbm_gbs", 6650.0), "measured"
+    return 1590.0, 1400.0, 6650.0, "fallback"
+
+
+def effective_flops(n, d, heads, nnz_blocks, causal=True):
+    qk = 2.0 * d * (n * (n + 1) / 2 if causal else n * n) * heads
+    return qk + (2.0 + 10.0) * d * BLOCK * BLOCK * nnz_blocks
+
+
+class ClockSampler:
+    """nvidia-smi samples during the timed region: SM clock, max clock, throttle reasons."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": max(mx), "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gen_inputs(seed, centres=CENTRES, run=0):
+    from adaptive_sparse_flash_b200 import inputs
+    return inputs.clustered(B, H, N, D, centres=centres, beta_q=BETA_Q, seed=seed, run=run)
+
+
+def cpu_baseline(arr):
+    """The float64 oracle on a bounded sample: one head, full forward + backward. Returns a dict."""
+    from oracle import attention as oa
+    t0 = time.perf_counter()
+    sub = {k: v[:1, :1] for k, v in arr.items()}
+    fw = oa.forward(sub["Q"], sub["K"], sub["V"], ALPHA, True)
+    oa.backward(sub["Q"], sub["K"], sub["V"], sub["dO"], ALPHA, True)
+    sec = time.perf_counter() - t0
+    nnz = int(fw["bits"].sum())
+    flops = effective_flops(N, D, 1, nnz)
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return {"value": flops / sec / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"head 0 of {H}: float64 oracle forward (all {N} rows) + backward (all rows and keys), "
+                      f"{sec:.1f} s, scaled by that head's effective FLOPs", "seconds": sec}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    arr = gen_inputs(seed=0)
+    times = []
+    for i in range(args.warmup + args.steps):
+        res = cpu_baseline(arr)
+        if i >= args.warmup:
+            times.append(res["seconds"])
+    sec = sum(times) / len(times)
+    val = res["value"] * res["seconds"] / sec
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": res["sample"]},
+            "cpu_baseline": {"kind": "oracle", "cores": res["cores"], "sample": res["sample"], "value": val,
+                             "unit": "TFLOP/s"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-sweep", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from adaptive_sparse_flash_b200 import binding as b
+    from adaptive_sparse_flash_b200 import build as bld
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    bld.build()
+    b.lib()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    arr = gen_inputs(seed=rank)
+    from adaptive_sparse_flash_b200 import inputs as _inputs
+    host = {k: torch.from_numpy(_inputs.bf16_bits(v).view(np.int16)).view(torch.bfloat16) for k, v in arr.items()}
+    dt = {k: v.to(dev) for k, v in host.items()}
+    Q, K, V, dO = dt["Q"], dt["K"], dt["V"], dt["dO"]
+    ws = b.alloc_workspace(B, H, N, D, device=dev)
+    opts = b.make_opts(ws)
+    O = torch.empty_like(Q)
+    tau = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    mask = torch.empty(b.mask_shape(B, H, N), dtype=torch.int32, device=dev)
+    dQ, dK, dV = (torch.empty(Q.shape, dtype=torch.float32, device=dev) for _ in range(3))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # larger than the 126 MB L2
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        b.entmax_attn_fwd(Q, K, V, O, tau, mask, ALPHA, True, opts, stream)
+        b.entmax_attn_bwd(Q, K, V, O, dO, tau, mask, dQ, dK, dV, ALPHA, True, opts, stream)
+
+    # warm-up, sparsity of this workload
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize(dev)
+    st = b.entmax_attn_check(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after warm-up: {b.entmax_status_str(st)}")
+    nnz = int(np.unpackbits(mask.cpu().numpy().view(np.uint8), bitorder="little").sum())
+    nqb = (N + BLOCK - 1) // BLOCK
+    causal_blocks = H * B * nqb * (nqb + 1) // 2
+    flops = effective_flops(N, D, B * H, nnz)
+
+    # timed region: per-step events (L2 flushed before each step, outside the events)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            b.entmax_attn_fwd(Q, K, V, O, tau, mask, ALPHA, True, opts, stream)
+            ev[i][1].record(stream)
+            b.entmax_attn_bwd(Q, K, V, O, dO, tau, mask, dQ, dK, dV, ALPHA, True, opts, stream)
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+    barrier()
+    st = b.entmax_attn_check(stream)
+    if st != 0:
+        raise RuntimeError(f"device status after timing: {b.entmax_status_str(st)}")
+    fwd_ms = [e0.elapsed_time(e1) for e0, e1, _ in ev]
+    bwd_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    step_ms = sum(f + g for f, g in zip(fwd_ms, bwd_ms)) / args.steps
+    step_ms = max_over_ranks(step_ms)
+    value = world * flops / (step_ms * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers (pinned), copies inside the timed region
+    pin = {k: v.pin_memory() for k, v in host.items()}
+    out_host = {k: torch.empty(Q.shape, dtype=torch.float32).pin_memory() for k in ("dQ", "dK", "dV")}
+    out_host["O"] = torch.empty(Q.shape, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pin.values())
+    d2h = sum(v.numel() * v.element_size() for v in out_host.values())
+    e2e_steps = max(2, min(args.steps, 5))
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        Q.copy_(pin["Q"], non_blocking=True)
+        K.copy_(pin["K"], non_blocking=True)
+        V.copy_(pin["V"], non_blocking=True)
+        dO.copy_(pin["dO"], non_blocking=True)
+        step()
+        out_host["dQ"].copy_(dQ, non_blocking=True)
+        out_host["dK"].copy_(dK, non_blocking=True)
+        out_host["dV"].copy_(dV, non_blocking=True)
+        out_host["O"].copy_(O, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+    e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12
+
+    # dense softmax baseline on the same inputs, same tiling
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    sdQ, sdK, sdV = (torch.empty(Q.shape, dtype=torch.float32, device=dev) for _ in range(3))
+    sopts = b.make_opts(ws)
+
+    def sm_step():
+        b.softmax_attn_fwd(Q, K, V, O, lse, True, None, stream)
+        b.softmax_attn_bwd(Q, K, V, O, dO, lse, sdQ, sdK, sdV, True, sopts, stream)
+
+    def timed(fn, reps):
+        fn()
+        torch.cuda.synchronize(dev)
+        tot = 0.0
+        for _ in range(reps):
+            flush.zero_()
+            a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            fn()
+            a1.record(stream)
+            torch.cuda.synchronize(dev)
+            tot += a0.elapsed_time(a1)
+        return tot / reps
+
+    softmax_ms = max_over_ranks(timed(sm_step, 3))
+
+    # roofline of the dominant kernel call (tensor-bound): algorithmic FLOPs per launch / its time
+    pk_burst, pk_sust, hbm, pk_kind = peaks()
+    f_ms, g_ms = sum(fwd_ms) / len(fwd_ms), sum(bwd_ms) / len(bwd_ms)
+    qk = 2.0 * D * N * (N + 1) / 2 * B * H
+    fwd_flops = qk + 2.0 * D * BLOCK * BLOCK * nnz
+    bwd_flops = 10.0 * D * BLOCK * BLOCK * nnz
+    if f_ms >= g_ms:
+        dom, dom_flops, dom_ms = "fwd_tc_kernel (entmax_attn_fwd)", fwd_flops, f_ms
+    else:
+        dom, dom_flops, dom_ms = "bwd_dkdv + bwd_dq (entmax_attn_bwd)", bwd_flops, g_ms
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
+                "frac": achieved / pk_sust, "traffic": None, "kernel": dom,
+                "peak_source": f"{pk_kind} bf16 sustained"}
+
+    # supplementary sweep: contiguous 128-token cluster runs, fewer centres = denser attention
+    sweep = []
+    if not args.no_sweep:
+        for c in (1, 2, 4, 8, 16):
+            a2 = gen_inputs(seed=100 + c, centres=c, run=128)
+            for k2, v2 in a2.items():
+                dt[k2].copy_(torch.from_numpy(v2).to(torch.bfloat16))
+            step()
+            torch.cuda.synchronize(dev)
+            nz = int(np.unpackbits(mask.cpu().numpy().view(np.uint8), bitorder="little").sum())
+            ms_e = timed(step, 3)
+            ms_s = timed(sm_step, 3)
+            fl = effective_flops(N, D, B * H, nz)
+            sweep.append({"centres": c, "block_sparsity": 1.0 - nz / causal_blocks, "entmax_ms": ms_e,
+                          "softmax_ms": ms_s, "eff_tflops": fl / (ms_e * 1e-3) / 1e12,
+                          "faster_than_dense": ms_e < ms_s})
+        for k2, v2 in arr.items():
+            dt[k2].copy_(torch.from_numpy(v2).to(torch.bfloat16))
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cpu = cpu_baseline(arr)
+        cpu.pop("seconds", None)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch_heads": B * H * world, "seq_len": N,
+                       "parallelism": f"independent heads x{world}" if world > 1 else "single GPU",
+                       "l2": "flushed before every timed step (256 MiB write)",
+                       "block_sparsity": 1.0 - nnz / causal_blocks, "nonzero_blocks": nnz,
+                       "fwd_ms": f_ms, "bwd_ms": g_ms, "softmax_fwd_bwd_ms": softmax_ms,
+                       "pct_bf16_peak": value / world / pk_sust * 100.0},
+            "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": 5 * args.steps,
+            "clocks": clk.summary(),
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "sparsity_sweep": sweep,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

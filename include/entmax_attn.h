@@ -95,8 +95,10 @@ entmax_status entmax_attn_fwd(const void* Q, const void* K, const void* V, void*
                               uint32_t* block_mask, int B, int H, int n, int d, float alpha, int causal,
                               entmax_dtype dt, const entmax_opts* opts, void* stream);
 
-/* Backward (bf16 only). Inputs are the forward's inputs and outputs and dO; the workspace must be the
- * one the forward filled. Outputs dQ, dK, dV: [B,H,n,d] bf16. Visits only the mask's nonzero blocks. */
+/* Backward (bf16 inputs only). Inputs are the forward's inputs and outputs and dO (bf16 [B,H,n,d]); the
+ * workspace must be the one the forward filled. Outputs dQ, dK, dV: float32 [B,H,n,d] (fp32 keeps
+ * large gradients exact to well below 1e-2; they are accumulated in fp32 TMEM). Visits only the
+ * mask's nonzero blocks. */
 entmax_status entmax_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                               const float* tau, const uint32_t* block_mask, void* dQ, void* dK, void* dV,
                               int B, int H, int n, int d, float alpha, int causal, entmax_dtype dt,
@@ -107,6 +109,7 @@ entmax_status entmax_attn_bwd(const void* Q, const void* K, const void* V, const
 entmax_status softmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* lse,
                                int B, int H, int n, int d, int causal, entmax_dtype dt,
                                const entmax_opts* opts, void* stream);
+/* softmax_attn_bwd: dQ, dK, dV float32 like entmax_attn_bwd; needs opts->workspace (same size query). */
 entmax_status softmax_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                                const float* lse, void* dQ, void* dK, void* dV, int B, int H, int n, int d,
                                int causal, entmax_dtype dt, const entmax_opts* opts, void* stream);

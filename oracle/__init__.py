@@ -18,6 +18,8 @@ What it computes, in plain float64 numpy:
   with bisection fallback, started from tau_h (same page, "Hybrid Solver &
   Sparsity-Awareness"; AdaSplash-2 technical summary, gist.science (hi),
   section 2, hybrid solver strategy).
+* `softmax.forward` / `softmax.backward`: dense softmax attention, the
+  reference for the in-library dense baseline.
 * `attention.forward` / `attention.backward`: entmax attention
   O = P V with s = Q K^T / sqrt(d), z = (alpha - 1) s, the bit-packed block
   mask (32 blocks per 32-bit word; gist.science (de), "Bit-Packed Block
@@ -29,4 +31,4 @@ against closed forms, brute force and finite differences; none is
 "parity unpinned".
 """
 
-from . import entmax, attention  # noqa: F401
+from . import entmax, attention, softmax  # noqa: F401

@@ -23,8 +23,10 @@ Mask"; gist.science (hi) technical summary, section 2, bit-packed block
 masking).
 
 Rows are independent in the forward, so they may be computed in chunks of
-rows; every sum over keys is taken whole. The key-side sums of dK and dV are
-matrix products accumulated over row chunks in float64.
+rows; every sum over keys is taken whole. p, u and dS vanish off the support
+{j : z_ij > tau_i}, so every sum that involves them runs over the support
+entries only (exact). The key-side sums of dK and dV accumulate over row
+chunks in float64.
 """
 from __future__ import annotations
 
@@ -32,7 +34,7 @@ import numpy as np
 
 from . import entmax
 
-__all__ = ["allowed", "scores", "forward", "backward", "block_mask", "pack_bits"]
+__all__ = ["allowed", "scores", "forward", "backward", "row_gradients", "block_mask", "pack_bits"]
 
 
 def allowed(rows: np.ndarray, n: int, causal: bool) -> np.ndarray:
@@ -49,18 +51,38 @@ def scores(q: np.ndarray, k: np.ndarray, scale: float) -> np.ndarray:
 
 
 def _row_forward(q, k, v, rows, alpha, causal, scale):
+    """Forward for query rows `rows` of one head.
+
+    The support S_i = {j : p_ij > 0} is kept as coordinate lists (rr, cc);
+    p, u and every product with them are summed over the support only,
+    which is exact because p_ij = u_ij = 0 off the support.
+    """
     n = k.shape[0]
     valid = allowed(rows, n, causal)
     z = (alpha - 1.0) * scores(q[rows], k, scale)
     tau = entmax.tau_bisect(z, valid, alpha)
-    p = entmax.probs(z, valid, tau, alpha)
     kk = 1.0 / (alpha - 1.0)
     x = np.where(valid, z - tau[:, None], 0.0)
-    sup = x > 0.0
-    u = np.where(sup, np.power(np.where(sup, x, 1.0), kk - 1.0), 0.0)
-    o = p @ np.asarray(v, np.float64)
-    obar = u @ np.asarray(v, np.float64)
-    return dict(z=z, valid=valid, tau=tau, p=p, u=u, O=o, Obar=obar, sum_u=u.sum(axis=1))
+    rr, cc = np.nonzero(x > 0.0)
+    xs = x[rr, cc]
+    p_s = np.power(xs, kk)
+    u_s = np.power(xs, kk - 1.0)
+    v64 = np.asarray(v, np.float64)
+    r = len(rows)
+    dv = v64.shape[1]
+    o = np.zeros((r, dv))
+    obar = np.zeros((r, dv))
+    np.add.at(o, rr, p_s[:, None] * v64[cc])
+    np.add.at(obar, rr, u_s[:, None] * v64[cc])
+    sum_u = np.bincount(rr, weights=u_s, minlength=r)
+    return dict(z=z, valid=valid, tau=tau, rr=rr, cc=cc, p_s=p_s, u_s=u_s, O=o, Obar=obar, sum_u=sum_u, n=n)
+
+
+def _dense(res, vals):
+    """Scatter support values into a dense [r, n] array."""
+    out = np.zeros((len(res["tau"]), res["n"]))
+    out[res["rr"], res["cc"]] = vals
+    return out
 
 
 def pack_bits(bits: np.ndarray) -> np.ndarray:
@@ -118,9 +140,8 @@ def forward(Q, K, V, alpha, causal, scale=None, block=64, rows=None, chunk=256):
                 Obar[b, h, sl] = res["Obar"]
                 tau[b, h, sl] = res["tau"]
                 sum_u[b, h, sl] = res["sum_u"]
-                pad = np.zeros((len(sel), nkb * block))
-                pad[:, :n] = res["p"]
-                bm = pad.reshape(len(sel), nkb, block).max(axis=2)
+                bm = np.zeros((len(sel), nkb))
+                np.maximum.at(bm, (res["rr"], res["cc"] // block), res["p_s"])
                 row_bmax[b, h, sl] = bm
                 row_bits[b, h, sl] = bm > 0.0
     out = dict(O=O, Obar=Obar, tau=tau, sum_u=sum_u, row_bits=row_bits, row_bmax=row_bmax,
@@ -139,6 +160,22 @@ def forward(Q, K, V, alpha, causal, scale=None, block=64, rows=None, chunk=256):
     return out
 
 
+def _row_backward(q, k, v, do, res, scale):
+    """delta, dS on the support, and dQ rows for one chunk (res from _row_forward)."""
+    rr, cc = res["rr"], res["cc"]
+    g_s = np.einsum("ij,ij->i", do[res_rows(res)][rr], v[cc])          # g_ij = dO_i . v_j on the support
+    r = len(res["tau"])
+    delta = np.bincount(rr, weights=res["u_s"] * g_s, minlength=r) / res["sum_u"]
+    ds_s = res["u_s"] * (g_s - delta[rr])
+    dq = np.zeros((r, q.shape[1]))
+    np.add.at(dq, rr, ds_s[:, None] * k[cc])
+    return delta, ds_s, scale * dq
+
+
+def res_rows(res):
+    return res["rows"]
+
+
 def backward(Q, K, V, dO, alpha, causal, scale=None, chunk=256, key_cols=None):
     """(dQ, dK, dV) in float64 for every (b, h).
 
@@ -151,9 +188,12 @@ def backward(Q, K, V, dO, alpha, causal, scale=None, chunk=256, key_cols=None):
     if scale is None:
         scale = 1.0 / np.sqrt(d)
     cols = np.arange(n) if key_cols is None else np.asarray(key_cols)
+    col_of = np.full(n, -1)
+    col_of[cols] = np.arange(len(cols))
+    dv_ = np.asarray(V).shape[-1]
     dQ = np.zeros((B, H, n, d))
     dK = np.zeros((B, H, len(cols), d))
-    dV = np.zeros((B, H, len(cols), d))
+    dV = np.zeros((B, H, len(cols), dv_))
     rows_all = np.arange(n)
     for b in range(B):
         for h in range(H):
@@ -164,13 +204,14 @@ def backward(Q, K, V, dO, alpha, causal, scale=None, chunk=256, key_cols=None):
             for c0 in range(0, n, chunk):
                 sel = rows_all[c0:c0 + chunk]
                 res = _row_forward(q, k, v, sel, alpha, causal, scale)
-                g = do[sel] @ v.T
-                u = res["u"]
-                delta = (u * g).sum(axis=1) / res["sum_u"]
-                ds = u * (g - delta[:, None])
-                dQ[b, h, sel] = scale * (ds @ k)
-                dK[b, h] += scale * (ds[:, cols].T @ q[sel])
-                dV[b, h] += res["p"][:, cols].T @ do[sel]
+                res["rows"] = sel
+                _, ds_s, dq = _row_backward(q, k, v, do, res, scale)
+                dQ[b, h, sel] = dq
+                rr, cc = res["rr"], res["cc"]
+                m = col_of[cc] >= 0                       # support entries in the requested columns
+                ci = col_of[cc[m]]
+                np.add.at(dK[b, h], ci, scale * ds_s[m][:, None] * q[sel][rr[m]])
+                np.add.at(dV[b, h], ci, res["p_s"][m][:, None] * do[sel][rr[m]])
     return dQ, dK, dV
 
 
@@ -189,8 +230,7 @@ def row_gradients(Q, K, V, dO, alpha, causal, rows, scale=None):
             v = np.asarray(V[b, h], np.float64)
             do = np.asarray(dO[b, h], np.float64)
             res = _row_forward(q, k, v, rows, alpha, causal, scale)
-            g = do[rows] @ v.T
-            delta = (res["u"] * g).sum(axis=1) / res["sum_u"]
-            ds = res["u"] * (g - delta[:, None])
-            dQ[b, h] = scale * (ds @ k)
+            res["rows"] = rows
+            _, _, dq = _row_backward(q, k, v, do, res, scale)
+            dQ[b, h] = dq
     return dQ

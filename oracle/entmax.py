@@ -77,10 +77,10 @@ def _candidates(z, valid, floor):
     counts = keep.sum(axis=1)
     c = max(int(counts.max()), 1)
     out = np.full((z.shape[0], c), -np.inf)
-    order = np.argsort(~keep, axis=1, kind="stable")[:, :c]
-    rows = np.arange(z.shape[0])[:, None]
-    sel = keep[rows, order]
-    out[sel] = z[rows, order][sel]
+    rr, cc = np.nonzero(keep)                  # row-major: entries of each row are contiguous
+    starts = np.concatenate([[0], np.cumsum(counts)[:-1]])
+    pos = np.arange(len(rr)) - starts[rr]
+    out[rr, pos] = z[rr, cc]
     return out
 
 
@@ -191,13 +191,24 @@ def histogram_tau(z, valid=None, alpha=1.5, bins=256, tol=1e-13):
 # Halley for alpha <= 1.5, Newton for 1.5 < alpha <= 2, secant above 2 (the
 # two pages disagree on alpha = 2 itself; Newton is used there, where f is
 # piecewise linear). A step that leaves the current bracket is replaced by
-# bisection. Stopping rule (not stated on the pages; reading): a row stops
-# when |f(tau)| <= ftol, or when a step moves tau by at most
-# xtol * max(1, |tau|), or after max_iter steps. The secant starts from the
-# two histogram bounds (tau_h, tau_H).
+# bisection.
+#
+# Readings where the pages are silent:
+#  * start: lo = max(tau_h, m - 1), hi = min(tau_h + w, m - n_i^(1-alpha)),
+#    first evaluation at lo; with the plain-bracket start (no histogram)
+#    lo = m - 1, hi = m - n_i^(1-alpha);
+#  * Halley / Newton stop when |f(tau)| <= ftol, or when a step moves tau by at
+#    most xtol * max(1, |tau|), or after max_iter steps;
+#  * the secant is the bracketing (Illinois) form: the first step is the
+#    secant through both bracket ends (f evaluated at both in one sweep), each
+#    later step the secant through the current ends, halving the f value of
+#    an end that is kept twice in a row; it stops when |f| <= ftol, when the
+#    bracket is narrower than xtol_bracket * max(1, |tau|) (about four float32
+#    ulps), or after max_iter steps.
 # ---------------------------------------------------------------------------
 
 HALLEY, NEWTON, SECANT = "halley", "newton", "secant"
+XTOL_BRACKET = 4.8e-7
 
 
 def method_for_alpha(alpha):
@@ -219,60 +230,93 @@ def _sums(zc, tau, k):
     return F0, F1, F2
 
 
-def hybrid_solve(z, valid=None, alpha=1.5, bins=256, ftol=1e-5, xtol=1e-6, max_iter=8):
+def hybrid_solve(z, valid=None, alpha=1.5, bins=256, ftol=1e-5, xtol=1e-6, max_iter=None, init="histogram"):
     """Returns (tau, steps, fallbacks) per row.
 
-    `steps` counts solver updates of tau after the histogram estimate;
-    `fallbacks` counts the updates that were bisection because the
-    method's step left the bracket.
+    `steps` counts solver updates of tau after the start; `fallbacks` counts
+    the updates that were bisection because the method's step left the
+    bracket (or was not finite).
     """
     z, valid = _as_rows(z, valid)
+    if max_iter is None:
+        max_iter = 12 if init == "histogram" else 24
     k = 1.0 / (alpha - 1.0)
-    w = 1.0 / (bins - 1)
     method = method_for_alpha(alpha)
-    m = row_max(z, valid)
     lo0, hi0 = bracket(z, valid, alpha)
-    tau_h, tau_H = histogram_tau(z, valid, alpha, bins)
     zc = _candidates(z, valid, lo0)
     r = z.shape[0]
-    lo = np.maximum(tau_h, lo0)
-    hi = np.minimum(tau_H, hi0)
-    bad = lo > hi
-    lo = np.where(bad, lo0, lo)
-    hi = np.where(bad, hi0, hi)
-    tau = lo.copy()
+    if init == "histogram":
+        tau_h, tau_H = histogram_tau(z, valid, alpha, bins)
+        lo = np.maximum(tau_h, lo0)
+        hi = np.minimum(tau_H, hi0)
+        bad = lo > hi
+        lo = np.where(bad, lo0, lo)
+        hi = np.where(bad, hi0, hi)
+    else:
+        lo, hi = lo0.copy(), hi0.copy()
     steps = np.zeros(r, dtype=np.int64)
     fallbacks = np.zeros(r, dtype=np.int64)
     done = np.zeros(r, dtype=bool)
-    prev_t = hi.copy()
-    prev_f = None
+
     if method == SECANT:
-        prev_f = _f(zc, prev_t, k)
-        # the upper point is a bracket end only if its sign says so
-        hi = np.where(prev_f <= 0.0, prev_t, hi0)
-        lo = np.where(prev_f > 0.0, np.maximum(lo, prev_t), lo)
+        flo = _f(zc, lo, k)
+        fhi = _f(zc, hi, k)
+        tau = lo.copy()
+        # an end whose sign contradicts the bracket is off only by rounding: accept it
+        stop_lo = (np.abs(flo) <= ftol) | (flo < 0.0)
+        stop_hi = ~stop_lo & ((np.abs(fhi) <= ftol) | (fhi > 0.0))
+        tau = np.where(stop_hi, hi, tau)
+        done = stop_lo | stop_hi
+        side = np.zeros(r, dtype=np.int64)
+        first = True
+        for _ in range(max_iter + 1):
+            if not first:
+                fc = _f(zc, tau, k)
+                conv = ~done & (np.abs(fc) <= ftol)
+                done |= conv
+                act = ~done
+                pos = fc > 0.0
+                up = act & pos
+                dn = act & ~pos
+                lo = np.where(up, tau, lo)
+                flo = np.where(up, fc, flo)
+                fhi = np.where(up & (side == 1), 0.5 * fhi, fhi)
+                hi = np.where(dn, tau, hi)
+                fhi = np.where(dn, fc, fhi)
+                flo = np.where(dn & (side == -1), 0.5 * flo, flo)
+                side = np.where(up, 1, np.where(dn, -1, side))
+            first = False
+            act = ~done & (steps < max_iter)
+            if not act.any():
+                break
+            with np.errstate(divide="ignore", invalid="ignore"):
+                cand = hi - fhi * (hi - lo) / (fhi - flo)
+            ok = np.isfinite(cand) & (cand > lo) & (cand < hi)
+            new = np.where(ok, cand, 0.5 * (lo + hi))
+            fallbacks += (act & ~ok).astype(np.int64)
+            steps += act.astype(np.int64)
+            tau = np.where(act, new, tau)
+            narrow = (hi - lo) <= XTOL_BRACKET * np.maximum(1.0, np.abs(tau))
+            done |= act & (narrow | (steps >= max_iter))
+        return tau, steps, fallbacks
+
+    tau = lo.copy()
     for _ in range(max_iter + 1):
         F0, F1, F2 = _sums(zc, tau, k)
         f = F0 - 1.0
-        stop = ~done & (np.abs(f) <= ftol)
-        done |= stop
+        done |= ~done & (np.abs(f) <= ftol)
         if np.all(done):
             break
         pos = f > 0.0
         lo = np.where(~done & pos, np.maximum(lo, tau), lo)
         hi = np.where(~done & ~pos, np.minimum(hi, tau), hi)
         fp = -k * F1
-        if method == HALLEY:
-            fpp = k * (k - 1.0) * F2
-            with np.errstate(divide="ignore", invalid="ignore"):
+        with np.errstate(divide="ignore", invalid="ignore"):
+            if method == HALLEY:
+                fpp = k * (k - 1.0) * F2
                 cand = tau - 2.0 * f * fp / (2.0 * fp * fp - f * fpp)
-        elif method == NEWTON:
-            with np.errstate(divide="ignore", invalid="ignore"):
+            else:
                 cand = tau - f / fp
-        else:
-            with np.errstate(divide="ignore", invalid="ignore"):
-                cand = tau - f * (tau - prev_t) / (f - prev_f)
-            prev_t, prev_f = tau.copy(), f.copy()
         ok = np.isfinite(cand) & (cand > lo) & (cand < hi)
         new = np.where(ok, cand, 0.5 * (lo + hi))
         active = ~done & (steps < max_iter)

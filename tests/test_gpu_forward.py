@@ -71,7 +71,10 @@ def test_fp32_path_causal(torch_cuda, alpha):
     arr = inputs.clustered(1, 2, 512, 64, centres=64, beta_q=4.0, seed=3, dtype="bf16", with_dO=False)
     ref = oa.forward(arr["Q"], arr["K"], arr["V"], alpha, causal=True, block=64)
     g = _run(torch_cuda, arr, alpha, True, torch_cuda.float32)
-    _check_all(g, ref, arr, alpha, True, 64, FP32_ABS * 10, None, f"fp32 path a={alpha}")
+    # alpha = 3 at |z| ~ 100: p = x^(1/2) turns the float32 rounding of z (~1e-5) into errors of a few 1e-3
+    # on near-threshold keys, so that case gets the bf16 bound; the others stay at 1e-3
+    tol = BF16_MAX_ABS if alpha > 2 else FP32_ABS * 10
+    _check_all(g, ref, arr, alpha, True, 64, tol, None, f"fp32 path a={alpha}")
 
 
 # ---- alpha sweep on the clustered generator (every solver branch) -----------------------------------------
