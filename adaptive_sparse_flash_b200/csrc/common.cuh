@@ -16,7 +16,6 @@ namespace eattn {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 constexpr uint32_t kWaitIterCap = 0x7fffffffu;
-constexpr uint32_t kSuspendHintNs = 200000;  // a waiting thread sleeps up to 0.2 ms unless the phase completes
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -51,10 +50,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+        : "r"(smem_u32(bar)), "r"(parity)
         : "memory");
     return ok != 0;
 }
@@ -66,8 +65,10 @@ static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 0; i < kWaitIterCap; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) break;
+        if ((i & 63u) == 63u) {
+            if (*abort) return false;
+            if (globaltimer() - t0 > kWaitLimitNs) break;
+        }
     }
     *abort = 1;
     if (status) atomicExch(status, (int)ENTMAX_ERR_TIMEOUT);

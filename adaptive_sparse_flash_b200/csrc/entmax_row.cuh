@@ -80,9 +80,10 @@ __device__ __forceinline__ void add_sums(float x, float k, float& F0, float& F1,
 }
 
 // ---------------------------------------------------------------------------------------------
-// Histogram ring (thread-owned row). hist: u32 [B slots][128 rows]. A 256-bit mask in registers
-// marks which slots hold a bin of the current window, so sliding the window clears bits instead of
-// shared memory, and the histogram needs no zeroing before use.
+// Histogram ring (thread-owned row). hist: u16 [B slots][128 rows], counts saturating at 65535 (a
+// saturated count only drops entries, which keeps the bound). A 256-bit mask in registers marks which
+// slots hold a bin of the current window, so sliding the window clears bits instead of shared memory,
+// and the histogram needs no zeroing before use.
 // ---------------------------------------------------------------------------------------------
 struct HistRow {
     float m_raw;    // running max of the raw score
@@ -136,7 +137,7 @@ __host__ __device__ __forceinline__ void live_clear(HistRow& h, int s0, int len,
 }
 
 // Raise the running max to `a_max` (raw) and slide the window.
-__device__ __forceinline__ void hist_raise(HistRow& h, float a_max, const SolveParams& sp, uint32_t* hist, int r) {
+__device__ __forceinline__ void hist_raise(HistRow& h, float a_max, const SolveParams& sp, uint16_t* hist, int r) {
     if (!(a_max > h.m_raw)) return;
     const int nt = bin_of(a_max, sp.cbin);
     const int B = sp.bins;
@@ -156,14 +157,15 @@ __device__ __forceinline__ void hist_raise(HistRow& h, float a_max, const SolveP
 }
 
 // Bin one raw score that passed a > thr_raw.
-__device__ __forceinline__ void hist_add(HistRow& h, float a, const SolveParams& sp, uint32_t* hist, int r) {
+__device__ __forceinline__ void hist_add(HistRow& h, float a, const SolveParams& sp, uint16_t* hist, int r) {
     const int b = bin_of(a, sp.cbin);
     const int j = h.top - b;
     if (j >= 0 && j < sp.bins) {
         const int s = b & (sp.bins - 1);
-        uint32_t* c = &hist[s * kTileRows + r];
+        uint16_t* c = &hist[s * kTileRows + r];
         if (slot_live(h, s)) {
-            *c += 1u;
+            const uint16_t v = *c;
+            if (v != 0xffffu) *c = (uint16_t)(v + 1u);
         } else {
             *c = 1u;
 #pragma unroll
@@ -173,12 +175,56 @@ __device__ __forceinline__ void hist_add(HistRow& h, float a, const SolveParams&
     }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Candidate stash (thread-owned row): raw scores of the entries binned while streaming, in shared
+// memory stash[i * 128 + r], i < kStashCap. Every entry of the final support is among them (it lies
+// above m - 1 >= m_run - 1), so the solver sums at any tau >= m_run - 1 can be taken over the stash
+// instead of another sweep over the keys. When the stash fills up, entries at or below the current
+// threshold are dropped; if it is still full the row is marked overflowed and falls back to sweeps.
+// ---------------------------------------------------------------------------------------------
+constexpr int kStashCap = 128;
+
+struct Stash {
+    int n;
+    bool overflow;
+};
+
+__device__ __forceinline__ void stash_add(Stash& st, float a, float thr_raw, float* stash, int r) {
+    if (st.overflow) return;
+    if (st.n == kStashCap) {
+        int j = 0;
+        for (int i = 0; i < kStashCap; ++i) {
+            const float v = stash[i * kTileRows + r];
+            if (v > thr_raw) stash[(j++) * kTileRows + r] = v;
+        }
+        st.n = j;
+        if (j == kStashCap) { st.overflow = true; return; }
+    }
+    stash[(st.n++) * kTileRows + r] = a;
+}
+
+// Solver sums over the stash at tau (and the secant's second point tau2 when `two`).
+template <int KIND>
+__device__ __forceinline__ void stash_sums(const Stash& st, const float* stash, int r, float cz, float k, float tau,
+                                           float tau2, bool two, float& F0, float& F1, float& F2, float& F0b) {
+    F0 = F1 = F2 = F0b = 0.f;
+    for (int i = 0; i < st.n; ++i) {
+        const float z = cz * stash[i * kTileRows + r];
+        const float x = z - tau;
+        if (x > 0.f) add_sums<KIND>(x, k, F0, F1, F2);
+        if (two) {
+            const float x2 = z - tau2;
+            if (x2 > 0.f) F0b += pow_k<KIND>(x2, k);
+        }
+    }
+}
+
 // Root tau_h of the left-edge binned function, in z units (a lower bound on tau*).
 // For k = 1 and k = 2 the root is found in closed form on its segment; for other k by a search over
 // the bin edges and then bisection inside the segment, keeping the end where f >= 0.
 // T[i] = i^k for i = 0..B (generic k only).
 template <int KIND>
-__device__ float hist_tau(const HistRow& h, const SolveParams& sp, const uint32_t* hist, int r, const float* T) {
+__device__ float hist_tau(const HistRow& h, const SolveParams& sp, const uint16_t* hist, int r, const float* T) {
     const int B = sp.bins;
     const float Bm1 = (float)(B - 1);
     auto cnt = [&](int j) -> float {

@@ -65,7 +65,8 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
     float* sK = reinterpret_cast<float*>(smem);                   // [64][D]
     float* sV = sK + kKeyBlk * D;                                  // [64][D]
     float* uni = sV + kKeyBlk * D;                                 // union: hist | O, U V accumulators
-    uint32_t* hist = reinterpret_cast<uint32_t*>(uni);             // [B][128]
+    uint16_t* hist = reinterpret_cast<uint16_t*>(uni);             // [B][128] u16
+    float* stash = uni + 256 * kTileRows / 2;                      // [kStashCap][128]
     float* sO = uni;                                               // [D][128]
     float* sOb = uni + D * kTileRows;                              // [D][128]
     const int uni_words = max(256 * kTileRows, 2 * D * kTileRows);
@@ -104,6 +105,9 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
     // ---- sweep 1: dense scores, running max, histogram, candidate blocks ----
     HistRow h;
     hist_init(h);
+    Stash sh;
+    sh.n = 0;
+    sh.overflow = false;
     for (int J = 0; J < nblk; ++J) {
         __syncthreads();
         stage<T, D>(sK, Kh, J * mb, mb, a.n);
@@ -119,19 +123,17 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
         bool any = false;
         if (sp.init_mode == 0) {
             hist_raise(h, amax, sp, hist, tid);
-            for (int jj = 0; jj < mb; ++jj)
-                if (sc[jj] > h.thr_raw) {
-                    any = true;
-                    hist_add(h, sc[jj], sp, hist, tid);
-                }
-        } else {
-            if (amax > h.m_raw) {
-                h.m_raw = amax;
-                h.thr_raw = amax - sp.inv_cz;
-                h.any = true;
-            }
-            for (int jj = 0; jj < mb; ++jj) any |= sc[jj] > h.thr_raw;
+        } else if (amax > h.m_raw) {
+            h.m_raw = amax;
+            h.thr_raw = amax - sp.inv_cz;
+            h.any = true;
         }
+        for (int jj = 0; jj < mb; ++jj)
+            if (sc[jj] > h.thr_raw) {
+                any = true;
+                if (sp.init_mode == 0) hist_add(h, sc[jj], sp, hist, tid);
+                stash_add(sh, sc[jj], h.thr_raw, stash, tid);
+            }
         if (any) atomicOr(&cand[J >> 5], 1u << (J & 31));
     }
 
@@ -143,6 +145,14 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
     if (!valid) s.done = true;
     if (valid && a.tau_hist) a.tau_hist[head + row] = tau_h;
     int sweeps = 1;
+    // rows whose candidates all fit the stash are solved on chip, with no further key sweep
+    if (valid && !sh.overflow) {
+        for (int it = 0; it < kMaxSweeps && !s.done; ++it) {
+            float F0, F1, F2, F0b;
+            stash_sums<KIND>(sh, stash, tid, sp.cz, sp.k, s.tau, s.tau2, s.need_two, F0, F1, F2, F0b);
+            solve_step(s, F0, F1, F2, F0b, sp);
+        }
+    }
 
     // ---- refinement sweep: solver sums only ----
     float last_step = INFINITY;
@@ -244,9 +254,11 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
 
     // refine while a row still takes steps wider than one bin; P V (also the check of sum p = 1);
     // if a tau moved, refine until every row stopped and finish with one more P V sweep
-    do {
-        refine_sweep();
-    } while (refine < kMaxSweeps && __syncthreads_or(!s.done && fabsf(last_step) > sp.w));
+    if (__syncthreads_or(!s.done)) {
+        do {
+            refine_sweep();
+        } while (refine < kMaxSweeps && __syncthreads_or(!s.done && fabsf(last_step) > sp.w));
+    }
     while (true) {
         const bool changed = pv_sweep();
         if (!changed || pv >= 3) break;

@@ -31,7 +31,8 @@ constexpr int BM = 128;           // query rows per tile
 constexpr int BN = 64;            // keys per block (= mask block)
 constexpr int NVS = 2;            // V ring stages
 constexpr int kThreads = 192;
-constexpr uint32_t kHistBytes = 256u * BM * 4u;  // 128 KB, reused for V / P / U after the dense sweep
+constexpr uint32_t kHistBytes = 256u * BM * 2u + kStashCap * BM * 4u;  // histogram + stash (128 KB), reused
+                                                                       // for V / P / U after the dense sweep
 
 template <int D>
 struct Cfg {
@@ -41,13 +42,16 @@ struct Cfg {
     static constexpr uint32_t kPBytes = BM * BN * 2;       // 16 KB
     static constexpr uint32_t offQ = 0;
     static constexpr uint32_t offK = offQ + kQBytes;
+    static constexpr int NPB = (D == 64) ? 2 : 1;          // P / U buffer sets
     static constexpr uint32_t offU = offK + NKS * kKBytes;  // union region
     static constexpr uint32_t offV = offU;                  // V ring inside the union
-    static constexpr uint32_t offP = offV + NVS * kKBytes;  // P buffers [2] (bf16 high part)
-    static constexpr uint32_t offPL = offP + 2 * kPBytes;   // P buffers [2] (bf16 low part)
-    static constexpr uint32_t offUU = offPL + 2 * kPBytes;  // U buffers [2]
-    static constexpr uint32_t offSmall = offU + kHistBytes;
-    static_assert(offUU + 2 * kPBytes <= offSmall, "union region too small");
+    static constexpr uint32_t offP = offV + NVS * kKBytes;  // P buffers [NPB] (bf16 high part)
+    static constexpr uint32_t offPL = offP + NPB * kPBytes; // P buffers [NPB] (bf16 low part)
+    static constexpr uint32_t offUU = offPL + NPB * kPBytes;  // U buffers [NPB] (bf16 high part)
+    static constexpr uint32_t offUL = offUU + NPB * kPBytes;  // U buffers [NPB] (bf16 low part)
+    static constexpr uint32_t kUnion =
+        (kHistBytes > NVS * kKBytes + 4 * NPB * kPBytes) ? kHistBytes : NVS * kKBytes + 4 * NPB * kPBytes;
+    static constexpr uint32_t offSmall = offU + kUnion;
     static constexpr uint32_t tmemCols = 512;
     static constexpr uint32_t colO = 128;
     static constexpr uint32_t colOb = 128 + D;
@@ -110,7 +114,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* plan_bits = reinterpret_cast<uint32_t*>(&sm + 1);  // [2][W]
     uint32_t* next = plan_bits + 2 * W;                          // [W]
     uint32_t* mrow = next + W;                                   // [2][W]
-    uint32_t* hist = reinterpret_cast<uint32_t*>(smem + C::offU);
+    uint16_t* hist = reinterpret_cast<uint16_t*>(smem + C::offU);                 // [256][128] u16, 64 KB
+    float* stash = reinterpret_cast<float*>(smem + C::offU + 256 * BM * 2);        // [kStashCap][128], 64 KB
 
     const SolveParams sp = a.sp;
     const int tid = threadIdx.x;
@@ -152,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sP0 = smem_u32(smem + C::offP);
     const uint32_t sPL0 = smem_u32(smem + C::offPL);
     const uint32_t sU0 = smem_u32(smem + C::offUU);
+    const uint32_t sUL0 = smem_u32(smem + C::offUL);
 
     if (warp == 5) {
         // ------------------------------------------------------------------ TMA issue
@@ -230,9 +236,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             auto issue_PV = [&](bool first) -> bool {
-                const uint32_t pb = pc & 1;
+                const uint32_t pb = pc % C::NPB;
                 const uint32_t vs = vc % NVS;
-                if (!wait_bounded(&sm.p_full[pb], (pc >> 1) & 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&sm.p_full[pb], (pc / C::NPB) & 1, abort_flag, a.status)) return false;
                 if (!wait_bounded(&sm.v_full[vs], (vc / NVS) & 1, abort_flag, a.status)) return false;
                 tc_fence_after();
                 const uint32_t vbase = sV0 + vs * C::kKBytes;
@@ -242,11 +248,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t dp = sdesc_sw128(sP0 + pb * C::kPBytes + kk * 32, 16, 1024);
                     const uint64_t dpl = sdesc_sw128(sPL0 + pb * C::kPBytes + kk * 32, 16, 1024);
                     const uint64_t du = sdesc_sw128(sU0 + pb * C::kPBytes + kk * 32, 16, 1024);
+                    const uint64_t dul = sdesc_sw128(sUL0 + pb * C::kPBytes + kk * 32, 16, 1024);
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-                    // P = P_hi + P_lo (two bf16 terms) keeps P V accurate to ~16 mantissa bits
+                    // P = P_hi + P_lo and U = U_hi + U_lo (two bf16 terms each) keep P V and U V accurate
+                    // to ~16 mantissa bits
                     mma_bf16_ss(tmem + C::colO, dp, dv, idPV, acc);
                     mma_bf16_ss(tmem + C::colO, dpl, dv, idPV, 1u);
                     mma_bf16_ss(tmem + C::colOb, du, dv, idPV, acc);
+                    mma_bf16_ss(tmem + C::colOb, dul, dv, idPV, 1u);
                 }
                 mma_commit(&sm.p_empty[pb]);
                 mma_commit(&sm.v_empty[vs]);
@@ -365,27 +374,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- sweep 0: dense ----
         HistRow h;
         hist_init(h);
+        Stash sh;
+        sh.n = 0;
+        sh.overflow = false;
         for (int J = 0; J < nblk && ok; ++J) {
             if (!(ok = load_S())) break;
             mask_S(J);
             const float amax = group_max();
-            bool any = false;
             if (sp.init_mode == 0) {
                 hist_raise(h, amax, sp, hist, r);
-                if (amax > h.thr_raw) {
-                    any = true;
+            } else if (amax > h.m_raw) {
+                h.m_raw = amax; h.thr_raw = amax - sp.inv_cz; h.any = true;
+            }
+            const bool any = amax > h.thr_raw;
+            if (any) {
 #pragma unroll
-                    for (int g = 0; g < 8; ++g) {
-                        if (gm[g] > h.thr_raw) {
+                for (int g = 0; g < 8; ++g) {
+                    if (gm[g] > h.thr_raw) {
 #pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                if (vbuf[8 * g + e] > h.thr_raw) hist_add(h, vbuf[8 * g + e], sp, hist, r);
+                        for (int e = 0; e < 8; ++e) {
+                            const float v = vbuf[8 * g + e];
+                            if (v > h.thr_raw) {
+                                if (sp.init_mode == 0) hist_add(h, v, sp, hist, r);
+                                stash_add(sh, v, h.thr_raw, stash, r);
+                            }
                         }
                     }
                 }
-            } else {
-                if (amax > h.m_raw) { h.m_raw = amax; h.thr_raw = amax - sp.inv_cz; h.any = true; }
-                any = amax > h.thr_raw;
             }
             const uint32_t ball = __ballot_sync(0xffffffffu, any);
             if (lane == 0 && ball) atomicOr(&next[J >> 5], 1u << (J & 31));
@@ -399,6 +414,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         solve_init(s, valid ? tau_h : 0.0f, valid ? m : 1.0f, n_i, sp);
         if (!valid) s.done = true;
         if (valid && a.tau_hist) a.tau_hist[head + row] = tau_h;
+        // rows whose candidates all fit the stash are solved on chip, with no further key sweep
+        if (ok && valid && !sh.overflow) {
+            for (int it = 0; it < kMaxSweeps && !s.done; ++it) {
+                float F0, F1, F2, F0b;
+                stash_sums<KIND>(sh, stash, r, sp.cz, sp.k, s.tau, s.tau2, s.need_two, F0, F1, F2, F0b);
+                solve_step(s, F0, F1, F2, F0b, sp);
+            }
+        }
 
         // ---- refinement sweep: solver sums at the current tau over the candidate blocks ----
         float last_step = INFINITY;
@@ -474,16 +497,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float amax = group_max();
                     const bool keep = sp.cz * amax > lo0;
                     const bool nz = sp.cz * amax - t > 0.f;
-                    const uint32_t pb = pc & 1;
+                    const uint32_t pb = pc % C::NPB;
                     ok = __all_sync(0xffffffffu,
-                                    wait_bounded(&sm.p_empty[pb], ((pc >> 1) & 1) ^ 1, abort_flag, a.status));
+                                    wait_bounded(&sm.p_empty[pb], ((pc / C::NPB) & 1) ^ 1, abort_flag, a.status));
                     if (!ok) break;
-                    const uint32_t pbase = sP0 + pb * Cfg<D>::kPBytes;
-                    const uint32_t plbase = sPL0 + pb * Cfg<D>::kPBytes;
-                    const uint32_t ubase = sU0 + pb * Cfg<D>::kPBytes;
+                    const uint32_t pbase = sP0 + pb * C::kPBytes;
+                    const uint32_t plbase = sPL0 + pb * C::kPBytes;
+                    const uint32_t ubase = sU0 + pb * C::kPBytes;
+                    const uint32_t ulbase = sUL0 + pb * C::kPBytes;
 #pragma unroll
                     for (int g = 0; g < 8; ++g) {
                         uint32_t ph[4] = {0u, 0u, 0u, 0u}, pl[4] = {0u, 0u, 0u, 0u}, uu[4] = {0u, 0u, 0u, 0u};
+                        uint32_t ul[4] = {0u, 0u, 0u, 0u};
                         if (sp.cz * gm[g] - t > 0.f) {
 #pragma unroll
                             for (int e = 0; e < 8; e += 2) {
@@ -516,13 +541,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const float2 hf = __bfloat1622float2(hi);
                                 ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hi);
                                 pl[e / 2] = pack_bf16x2(pv2[0] - hf.x, pv2[1] - hf.y);
-                                uu[e / 2] = pack_bf16x2(uv2[0], uv2[1]);
+                                const __nv_bfloat162 uh = __floats2bfloat162_rn(uv2[0], uv2[1]);
+                                const float2 uf = __bfloat1622float2(uh);
+                                uu[e / 2] = *reinterpret_cast<const uint32_t*>(&uh);
+                                ul[e / 2] = pack_bf16x2(uv2[0] - uf.x, uv2[1] - uf.y);
                             }
                         }
                         const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)g);
                         st_shared_v4(pbase + off, ph[0], ph[1], ph[2], ph[3]);
                         st_shared_v4(plbase + off, pl[0], pl[1], pl[2], pl[3]);
                         st_shared_v4(ubase + off, uu[0], uu[1], uu[2], uu[3]);
+                        st_shared_v4(ulbase + off, ul[0], ul[1], ul[2], ul[3]);
                     }
                     fence_proxy_async_smem();
                     mbar_arrive(&sm.p_full[pb]);
@@ -546,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Schedule: refine while some row still takes steps wider than one bin; then P V, whose sums
         // double as the check of sum p = 1. If any tau still moved, refine until every row has
         // stopped (cheaper than repeated P V sweeps) and finish with one more P V sweep.
-        if (ok) {
+        if (ok && bar_or_compute(!s.done)) {
             do {
                 refine_sweep();
             } while (ok && refine < kMaxSweeps &&

@@ -40,7 +40,7 @@ struct BarsS {
     uint64_t kv_full[NST], kv_empty[NST];
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full[2], p_empty[2];
-    uint64_t pv_done, o_full, drain;
+    uint64_t pv_done[2], o_full, drain;  // pv_done[j & 1]: P V of block j has completed
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -82,7 +82,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bb.s_full[i], 1); mbar_init(&bb.s_empty[i], BM);
             mbar_init(&bb.p_full[i], BM); mbar_init(&bb.p_empty[i], 1);
         }
-        mbar_init(&bb.pv_done, 1);
+        mbar_init(&bb.pv_done[0], 1);
+        mbar_init(&bb.pv_done[1], 1);
         mbar_init(&bb.o_full, 1);
         mbar_init(&bb.drain, 1);
         bb.abort_flag = 0;
@@ -155,7 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 sdesc_sw128(vb + kk * 2048, BN * 128, 1024), idPV, (J > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&bb.p_empty[pb]);
                 mma_commit(&bb.kv_empty[st]);
-                mma_commit(&bb.pv_done);
+                mma_commit(&bb.pv_done[J & 1]);
                 return true;
             };
             if (ok) ok = issue_S(0);
@@ -203,11 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float m_new = resc ? bm : m_used;
                 const float f = (resc && m_used != -INFINITY) ? exp2f(m_used - m_new) : 1.f;
                 if (J > 0 && __any_sync(0xffffffffu, f != 1.f)) {
-                    // O holds P V of blocks < J: wait for those MMAs, then scale this warp's rows
-                    bool w1 = true;
-                    if (J >= 2) w1 = wait_bounded(&bb.pv_done, (J - 2) & 1, abort_flag, a.status);
-                    w1 = w1 && wait_bounded(&bb.pv_done, (J - 1) & 1, abort_flag, a.status);
-                    ok = __all_sync(0xffffffffu, w1);
+                    // O holds P V of blocks < J: wait for P V (J-1) (MMAs complete in issue order), then
+                    // scale this warp's rows. Each pv_done barrier is at most one phase behind here.
+                    ok = __all_sync(0xffffffffu, wait_bounded(&bb.pv_done[(J - 1) & 1], ((J - 1) >> 1) & 1,
+                                                              abort_flag, a.status));
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll

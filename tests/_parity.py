@@ -50,3 +50,38 @@ def check_mask(mask_gpu_words, bits_ref, bmax_ref, where=""):
     bad = (g != bits_ref) & ~(bmax_ref < MASK_EXEMPT_P)
     assert not bad.any(), f"{where}: {int(bad.sum())} mask bits differ (of {bits_ref.size})"
     return int((g != bits_ref).sum())
+
+
+def conditioning(arr, alpha, causal, xmin=1e-2, flip=0.0):
+    """Rows with an entry close to the support boundary, and the key columns those rows touch.
+
+    A row is flagged when some support entry has 0 < z - tau* < xmin, or when some allowed entry has
+    |z - tau*| < flip * max(1, |tau*|). For alpha > 2, u = (z - tau)^(k-1) grows without bound as
+    z - tau -> 0 and p = (z - tau)^k has an unbounded slope, so the float32 rounding of the scores
+    (~1e-7 |z|) moves such entries by amounts no float32 score can resolve; for alpha = 2, u is the
+    support indicator and an entry within rounding of tau* can land on either side. These rows and
+    columns are reported and left out of the comparison they cannot meet.
+    Returns (bad_rows[B,H,n] bool, bad_cols[B,H,n] bool).
+    """
+    from oracle import attention as oa
+    from oracle import entmax as oe
+    Q, K = arr["Q"], arr["K"]
+    B, H, n, d = Q.shape
+    bad_rows = np.zeros((B, H, n), bool)
+    bad_cols = np.zeros((B, H, n), bool)
+    for b in range(B):
+        for h in range(H):
+            for c0 in range(0, n, 512):
+                rows = np.arange(c0, min(n, c0 + 512))
+                valid = oa.allowed(rows, n, causal)
+                z = (alpha - 1) * oa.scores(Q[b, h][rows], K[b, h], 1 / np.sqrt(d))
+                tau = oe.tau_bisect(z, valid, alpha)
+                x = np.where(valid, z - tau[:, None], -1.0)
+                sup = x > 0
+                near = sup & (x < xmin)
+                if flip > 0:
+                    near |= valid & (np.abs(z - tau[:, None]) < flip * np.maximum(1.0, np.abs(tau))[:, None])
+                br = near.any(axis=1)
+                bad_rows[b, h, rows] = br
+                bad_cols[b, h] |= sup[br].any(axis=0)
+    return bad_rows, bad_cols
