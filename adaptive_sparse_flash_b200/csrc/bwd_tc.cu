@@ -246,7 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int I = w * 32 + __ffs(bits) - 1;
                     bits &= bits - 1;
                     const uint32_t st = i & 1;
-                    if (!(ok = wait_bounded(&bb.q_empty[st], ((i >> 1) & 1) ^ 1, abort_flag, a.status))) break;
+                    if (!(ok = wait_bounded(&bb.q_empty[st], ((i >> 1) & 1) ^ 1, abort_flag, a.status, true))) break;
                     unsigned char* base = smem + C::offSt + st * C::kStage;
                     mbar_arrive_expect_tx(&bb.q_full[st], 2 * C::kBlk + 512);
                     for (int c = 0; c < D / 64; ++c) {
@@ -267,13 +267,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16_f32(TM, TB, false, false);   // K Q^T, V dO^T
             constexpr uint32_t idG = idesc_bf16_f32(TM, D, false, true);     // P^T dO, dS^T Q (MN-major B)
-            bool ok = wait_bounded(&bb.kv_full, 0, abort_flag, a.status);
+            bool ok = wait_bounded(&bb.kv_full, 0, abort_flag, a.status, true);
             tc_fence_after();
             uint32_t i = 0;
             auto issue_S = [&](uint32_t idx) -> bool {
                 const uint32_t st = idx & 1, sb = idx & 1;
-                if (!wait_bounded(&bb.q_full[st], (idx >> 1) & 1, abort_flag, a.status)) return false;
-                if (!wait_bounded(&bb.s_empty[sb], ((idx >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&bb.q_full[st], (idx >> 1) & 1, abort_flag, a.status, true)) return false;
+                if (!wait_bounded(&bb.s_empty[sb], ((idx >> 1) & 1) ^ 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t qb = sSt + st * C::kStage, ob = qb + C::kBlk;
 #pragma unroll
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto issue_G = [&](uint32_t idx, bool first) -> bool {
                 const uint32_t st = idx & 1;
-                if (!wait_bounded(&bb.ds_full, idx & 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&bb.ds_full, idx & 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t qb = sSt + st * C::kStage, ob = qb + C::kBlk;
 #pragma unroll
@@ -527,7 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int J = w * 32 + __ffs(bits) - 1;
                     bits &= bits - 1;
                     const uint32_t st = i & 1;
-                    if (!(ok = wait_bounded(&bb.q_empty[st], ((i >> 1) & 1) ^ 1, abort_flag, a.status))) break;
+                    if (!(ok = wait_bounded(&bb.q_empty[st], ((i >> 1) & 1) ^ 1, abort_flag, a.status, true))) break;
                     unsigned char* base = smem + C::offSt + st * C::kStage;
                     mbar_arrive_expect_tx(&bb.q_full[st], 2 * C::kBlk);
                     for (int c = 0; c < D / 64; ++c) {
@@ -546,12 +546,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16_f32(TM, TB, false, false);   // Q K^T, dO V^T
             constexpr uint32_t idG = idesc_bf16_f32(TM, D, false, true);     // dS K (MN-major B)
-            bool ok = wait_bounded(&bb.kv_full, 0, abort_flag, a.status);
+            bool ok = wait_bounded(&bb.kv_full, 0, abort_flag, a.status, true);
             tc_fence_after();
             auto issue_S = [&](uint32_t idx) -> bool {
                 const uint32_t st = idx & 1, sb = idx & 1;
-                if (!wait_bounded(&bb.q_full[st], (idx >> 1) & 1, abort_flag, a.status)) return false;
-                if (!wait_bounded(&bb.s_empty[sb], ((idx >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&bb.q_full[st], (idx >> 1) & 1, abort_flag, a.status, true)) return false;
+                if (!wait_bounded(&bb.s_empty[sb], ((idx >> 1) & 1) ^ 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t kb = sSt + st * C::kStage, vb = kb + C::kBlk;
 #pragma unroll
@@ -569,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto issue_G = [&](uint32_t idx, bool first) -> bool {
                 const uint32_t st = idx & 1;
-                if (!wait_bounded(&bb.ds_full, idx & 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&bb.ds_full, idx & 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t kb = sSt + st * C::kStage;
 #pragma unroll

@@ -60,10 +60,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity. Returns false (and sets *abort) on timeout or
 // when another role of the CTA has already aborted.
-static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort, int* status) {
+// `backoff`: the waiting thread sleeps between polls (exponentially, up to 256 ns), for the issuing warps
+// whose spinning would otherwise take issue slots from the compute warps on the same scheduler.
+static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                                 bool backoff = false) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
+    uint32_t ns = 8;
     for (uint32_t i = 0; i < kWaitIterCap; ++i) {
+        if (backoff) {
+            __nanosleep(ns);
+            ns = ns < 256 ? 2 * ns : 256;
+        }
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 63u) {
             if (*abort) return false;
@@ -139,6 +147,25 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (M x 16 bf16 per instruction) read from tensor memory, one row
+// per lane, two bf16 per 32-bit column (element 2j in the low half).
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 8 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+                 "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // Arrive on `bar` once every tcgen05 op issued so far by this thread has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

@@ -80,24 +80,29 @@ __device__ __forceinline__ void add_sums(float x, float k, float& F0, float& F1,
 }
 
 // ---------------------------------------------------------------------------------------------
-// Histogram ring (thread-owned row). hist: u16 [B slots][128 rows], counts saturating at 65535 (a
-// saturated count only drops entries, which keeps the bound). A 256-bit mask in registers marks which
-// slots hold a bin of the current window, so sliding the window clears bits instead of shared memory,
-// and the histogram needs no zeroing before use.
+// Histogram ring (thread-owned row).
+//   hist  u16 [B slots][128 rows]; counts saturate at 65535 (a saturated count only drops entries,
+//         which keeps the bound);
+//   live  u32 [128 rows][kLiveStride]: bit s of row r's 8 words marks slot s as holding a counted bin
+//         of the current window. Sliding the window clears bits instead of counts, so the histogram
+//         needs no zeroing and a slide costs a few word operations.
 // ---------------------------------------------------------------------------------------------
+constexpr int kLiveStride = 9;  // words per row (8 used; odd stride keeps rows on distinct banks)
+
 struct HistRow {
-    float m_raw;    // running max of the raw score
-    float thr_raw;  // raw threshold for binning: z > m_run - 1
-    int top;        // bin index of the running max
-    bool any;       // any entry seen
-    uint32_t live[8];  // slot s holds a counted bin of the window iff bit s of live is set
+    float m_raw;     // running max of the raw score
+    float thr_raw;   // raw threshold for binning: z > m_run - 1
+    int top;         // bin index of the running max
+    bool any;        // any entry seen
+    uint32_t* live;  // this row's live words in shared memory
 };
 
-__device__ __forceinline__ void hist_init(HistRow& h) {
+__device__ __forceinline__ void hist_init(HistRow& h, uint32_t* live_all, int r) {
     h.m_raw = -INFINITY;
     h.thr_raw = INFINITY;
     h.top = 0;
     h.any = false;
+    h.live = live_all + r * kLiveStride;
 #pragma unroll
     for (int i = 0; i < 8; ++i) h.live[i] = 0u;
 }
@@ -107,70 +112,59 @@ __device__ __forceinline__ int bin_of(float a, float cbin) {
     return __float2int_rd(y);
 }
 
-__device__ __forceinline__ bool slot_live(const HistRow& h, int s) {
-    uint32_t w = 0u;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w = (i == (s >> 5)) ? h.live[i] : w;
-    return (w >> (s & 31)) & 1u;
-}
-
-// Clear the live bits of the `len` slots starting at slot `s0` (circular over B slots, len < B).
-__host__ __device__ __forceinline__ void live_clear(HistRow& h, int s0, int len, int B) {
-    // bits [s0, s0 + len) of a B-bit ring; B <= 256 and a power of two
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int lo = i * 32;
-        if (lo >= B) break;
-        // positions p in [lo, lo+32) with (p - s0) mod B < len
-        uint32_t m = 0u;
-        const int a0 = ((lo - s0) % B + B) % B;  // offset of bit 0 of this word from s0
-        if (a0 < len) m = (len - a0 >= 32) ? 0xffffffffu : ((1u << (len - a0)) - 1u);
-        // the run may wrap into the top of this word
-        const int wrap = a0 + 32 - B;  // bits of this word whose offset wrapped past B
-        if (wrap > 0) {
-            const int first = 32 - wrap;  // bit index where offset wraps to 0
-            const int cnt = min(wrap, len);
-            if (cnt > 0) m |= ((cnt >= 32) ? 0xffffffffu : ((1u << cnt) - 1u)) << first;
-        }
-        h.live[i] &= ~m;
+// Bits [s0, s0 + len) of a B-bit ring (B <= 256, a power of two, len < B) as 8 words (host-testable).
+__host__ __device__ __forceinline__ uint32_t ring_word_mask(int i, int s0, int len, int B) {
+    const int lo = i * 32;
+    if (lo >= B) return 0u;
+    uint32_t m = 0u;
+    const int a0 = (lo - s0) & (B - 1);  // offset of bit 0 of this word from s0
+    if (a0 < len) m = (len - a0 >= 32) ? 0xffffffffu : ((1u << (len - a0)) - 1u);
+    const int wrap = a0 + 32 - B;  // bits of this word whose offset wrapped past B
+    if (wrap > 0) {
+        const int cnt = min(wrap, len);
+        if (cnt > 0) m |= ((cnt >= 32) ? 0xffffffffu : ((1u << cnt) - 1u)) << (32 - wrap);
     }
+    return m;
 }
 
 // Raise the running max to `a_max` (raw) and slide the window.
-__device__ __forceinline__ void hist_raise(HistRow& h, float a_max, const SolveParams& sp, uint16_t* hist, int r) {
+__device__ __forceinline__ void hist_raise(HistRow& h, float a_max, float cbin, float inv_cz, int B) {
     if (!(a_max > h.m_raw)) return;
-    const int nt = bin_of(a_max, sp.cbin);
-    const int B = sp.bins;
+    const int nt = bin_of(a_max, cbin);
     if (h.any && nt > h.top) {
         const int d = nt - h.top;
         if (d >= B) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) h.live[i] = 0u;
         } else {
-            live_clear(h, (h.top + 1) & (B - 1), d, B);
+            const int s0 = (h.top + 1) & (B - 1);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t m = ring_word_mask(i, s0, d, B);
+                if (m) h.live[i] &= ~m;
+            }
         }
     }
     h.top = h.any ? max(h.top, nt) : nt;
     h.any = true;
     h.m_raw = a_max;
-    h.thr_raw = a_max - sp.inv_cz;
+    h.thr_raw = a_max - inv_cz;
 }
 
 // Bin one raw score that passed a > thr_raw.
-__device__ __forceinline__ void hist_add(HistRow& h, float a, const SolveParams& sp, uint16_t* hist, int r) {
-    const int b = bin_of(a, sp.cbin);
+__device__ __forceinline__ void hist_add(const HistRow& h, float a, float cbin, int B, uint16_t* hist, int r) {
+    const int b = bin_of(a, cbin);
     const int j = h.top - b;
-    if (j >= 0 && j < sp.bins) {
-        const int s = b & (sp.bins - 1);
+    if (j >= 0 && j < B) {
+        const int s = b & (B - 1);
         uint16_t* c = &hist[s * kTileRows + r];
-        if (slot_live(h, s)) {
+        const uint32_t w = h.live[s >> 5], bit = 1u << (s & 31);
+        if (w & bit) {
             const uint16_t v = *c;
             if (v != 0xffffu) *c = (uint16_t)(v + 1u);
         } else {
             *c = 1u;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (i == (s >> 5)) h.live[i] |= 1u << (s & 31);
+            h.live[s >> 5] = w | bit;
         }
     }
 }
@@ -180,9 +174,10 @@ __device__ __forceinline__ void hist_add(HistRow& h, float a, const SolveParams&
 // memory stash[i * 128 + r], i < kStashCap. Every entry of the final support is among them (it lies
 // above m - 1 >= m_run - 1), so the solver sums at any tau >= m_run - 1 can be taken over the stash
 // instead of another sweep over the keys. When the stash fills up, entries at or below the current
-// threshold are dropped; if it is still full the row is marked overflowed and falls back to sweeps.
+// threshold are dropped; if that leaves it more than half full, the row is marked overflowed (it falls
+// back to sweeps) so that the pruning work stays amortised O(1) per entry.
 // ---------------------------------------------------------------------------------------------
-constexpr int kStashCap = 128;
+constexpr int kStashCap = 64;
 
 struct Stash {
     int n;
@@ -198,9 +193,26 @@ __device__ __forceinline__ void stash_add(Stash& st, float a, float thr_raw, flo
             if (v > thr_raw) stash[(j++) * kTileRows + r] = v;
         }
         st.n = j;
-        if (j == kStashCap) { st.overflow = true; return; }
+        if (j > kStashCap / 2) { st.overflow = true; return; }
     }
     stash[(st.n++) * kTileRows + r] = a;
+}
+
+// Bin every stash entry above thr_raw into a histogram whose window top is the bin of m_raw (the row's
+// running max so far). Used once per row: at the end of the dense sweep, or when the stash overflows and
+// the row switches to streaming the histogram.
+__device__ __forceinline__ void hist_from_stash(HistRow& h, const Stash& st, const float* stash, float m_raw,
+                                                float thr_raw, float cbin, int B, uint16_t* hist, int r) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h.live[i] = 0u;
+    h.any = m_raw > -INFINITY;
+    h.m_raw = m_raw;
+    h.thr_raw = thr_raw;
+    h.top = h.any ? bin_of(m_raw, cbin) : 0;
+    for (int i = 0; i < st.n; ++i) {
+        const float v = stash[i * kTileRows + r];
+        if (v > thr_raw) hist_add(h, v, cbin, B, hist, r);
+    }
 }
 
 // Solver sums over the stash at tau (and the secant's second point tau2 when `two`).
@@ -220,51 +232,114 @@ __device__ __forceinline__ void stash_sums(const Stash& st, const float* stash, 
 }
 
 // Root tau_h of the left-edge binned function, in z units (a lower bound on tau*).
-// For k = 1 and k = 2 the root is found in closed form on its segment; for other k by a search over
-// the bin edges and then bisection inside the segment, keeping the end where f >= 0.
-// T[i] = i^k for i = 0..B (generic k only).
+// For k = 1 and k = 2 the root is found in closed form on its segment (exact integer moments); for
+// other k by a search over the bin edges and then bisection inside the segment, keeping the end where
+// f >= 0. T[i] = i^k for i = 0..B (generic k only). The result is lowered by a few float32 ulps so that
+// rounding cannot lift it above the binned root.
 template <int KIND>
-__device__ float hist_tau(const HistRow& h, const SolveParams& sp, const uint16_t* hist, int r, const float* T) {
+__host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, const uint16_t* hist, int r, const float* T) {
     const int B = sp.bins;
     const float Bm1 = (float)(B - 1);
-    auto cnt = [&](int j) -> float {
+    auto cnt = [&](int j) -> uint32_t {
         const int sl = (h.top - j) & (B - 1);
-        return slot_live(h, sl) ? (float)hist[sl * kTileRows + r] : 0.0f;
+        return ((h.live[sl >> 5] >> (sl & 31)) & 1u) ? (uint32_t)hist[sl * kTileRows + r] : 0u;
     };
+    float tau_h;
     if constexpr (KIND == kAlpha15 || KIND == kAlpha2) {
-        // A0 = sum c_j, A1 = sum c_j (J - j), A2 = sum c_j (J - j)^2 over offsets j < J (exact integers)
-        double A0 = 0.0, A1 = 0.0, A2 = 0.0;
-        const double thr = (KIND == kAlpha15) ? (double)Bm1 * (double)Bm1 : (double)Bm1;
-        int J = 1;
-        for (; J < B; ++J) {
-            if (J > 1) {
-                A2 += 2.0 * A1 + A0;
-                A1 += A0;
+        // A0 = sum c_j, A1 = sum c_j (J - j), A2 = sum c_j (J - j)^2 over offsets j < J (exact integers).
+        // Only live bins are visited (set bits of the live mask, in order of offset j = top - bin); between
+        // them the moments move in closed form, and the first J at which the binned function reaches 0
+        // (A2 >= (B-1)^2, or A1 >= B-1 for k = 1) is found by a float estimate corrected in integers.
+        long long A0 = 0, A1 = 0, A2 = 0;
+        const long long thr = (KIND == kAlpha15) ? (long long)(B - 1) * (B - 1) : (long long)(B - 1);
+        auto Ak = [&](long long t) -> long long {  // A_k(J0 + t) from the moments at J0
+            return (KIND == kAlpha15) ? A2 + 2 * t * A1 + t * t * A0 : A1 + t * A0;
+        };
+        auto first_cross = [&]() -> long long {  // smallest t >= 1 with A_k(J0 + t) >= thr (A0 > 0)
+            float tf;
+            if constexpr (KIND == kAlpha15) {
+                const float a0 = (float)A0, a1 = (float)A1, d2 = (float)(A2 - thr);
+                tf = (-a1 + sqrtf(fmaxf(a1 * a1 - a0 * d2, 0.0f))) / a0;
+            } else {
+                tf = (float)(thr - A1) / (float)A0;
             }
-            const double c = (double)cnt(J - 1);
-            A0 += c;
-            A1 += c;
-            A2 += c;
-            const double F = (KIND == kAlpha15) ? A2 : A1;
-            if (F >= thr) break;
+            long long t = (long long)fmaxf(1.0f, ceilf(tf));
+            while (t > 1 && Ak(t - 1) >= thr) --t;
+            while (Ak(t) < thr) ++t;
+            return t;
+        };
+        uint32_t lw[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) lw[i] = h.live[i];
+        const int stop = h.top & (B - 1);
+        const int nw = B >= 32 ? B / 32 : 1;
+        int J = B - 1, J0 = 0;  // moments are evaluated at J0 (bins with offset < J0)
+        bool found = false;
+        // visit slots stop, stop-1, ..., 0, B-1, ..., stop+1: word by word from the word holding `stop`
+        for (int step = 0; step <= nw && !found; ++step) {
+            const int wi = ((stop >> 5) - step + 2 * nw) % nw;
+            uint32_t bits = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) bits = (i == wi) ? lw[i] : bits;
+            if (B < 32) bits &= (1u << B) - 1u;
+            if (step == 0) bits &= (stop & 31) == 31 ? 0xffffffffu : ((2u << (stop & 31)) - 1u);   // slots <= stop
+            if (step == nw) bits &= (stop & 31) == 31 ? 0u : ~((2u << (stop & 31)) - 1u);        // slots > stop
+            while (bits && !found) {
+#ifdef __CUDA_ARCH__
+                const int bpos = 31 - __clz(bits);
+#else
+                const int bpos = 31 - __builtin_clz(bits);
+#endif
+                bits &= ~(1u << bpos);
+                const int sl = wi * 32 + bpos;
+                const long long c = hist[sl * kTileRows + r];
+                if (c == 0) continue;
+                const int jn = (stop - sl) & (B - 1);  // offset of this bin below the top
+                const int J1 = jn + 1;                 // first J at which the bin counts
+                if (A0 > 0) {
+                    const long long t = first_cross();
+                    if (J0 + t < J1) {  // crosses before this bin starts to count
+                        A2 = (KIND == kAlpha15) ? Ak(t) : A2;
+                        A1 += t * A0;
+                        J = J0 + (int)t;
+                        found = true;
+                        break;
+                    }
+                    const long long T = J1 - J0;
+                    A2 += 2 * T * A1 + T * T * A0;
+                    A1 += T * A0;
+                }
+                A0 += c;
+                A1 += c;
+                A2 += c;
+                J0 = J1;
+                if (((KIND == kAlpha15) ? A2 : A1) >= thr) { J = J1; found = true; }
+            }
+        }
+        if (!found && A0 > 0) {
+            const long long t = first_cross();
+            A2 = (KIND == kAlpha15) ? Ak(t) : A2;
+            A1 += t * A0;
+            J = J0 + (int)t;
         }
         if (J >= B) J = B - 1;
-        double u;  // tau_h = (top - J + u) w, u in [0, 1)
+        float u;  // tau_h = (top - J + u) w, u in [0, 1)
+        const float a0 = (float)A0, a1 = (float)A1, a2 = (float)A2;
         if constexpr (KIND == kAlpha15) {
-            const double disc = fmax(A1 * A1 - A0 * (A2 - thr), 0.0);
-            u = (A1 - sqrt(disc)) / A0;
+            const float disc = fmaxf(a1 * a1 - a0 * (a2 - (float)thr), 0.0f);
+            u = (a1 - sqrtf(disc)) / a0;
         } else {
-            u = (A1 - thr) / A0;
+            u = (a1 - (float)thr) / a0;
         }
-        u = fmin(fmax(u, 0.0), 1.0);
-        return (float)(((double)(h.top - J) + u) * (double)sp.w);
+        u = fminf(fmaxf(u, 0.0f), 1.0f);
+        tau_h = ((float)(h.top - J) + u) * sp.w;
     } else {
         const float thr = T[B - 1];
         auto F = [&](int J) -> float {
             float s = 0.0f;
             for (int j = 0; j < J; ++j) {
-                const float c = cnt(j);
-                if (c != 0.0f) s = fmaf(c, T[J - j], s);
+                const uint32_t c = cnt(j);
+                if (c) s = fmaf((float)c, T[J - j], s);
             }
             return s;
         };
@@ -281,14 +356,19 @@ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, const uint16_
             const float um = 0.5f * (ulo + uhi);
             float s = 0.0f;
             for (int j = 0; j < J; ++j) {
-                const float c = cnt(j);
+                const uint32_t c = cnt(j);
                 const float x = (float)(J - j) - um;
-                if (c != 0.0f && x > 0.0f) s = fmaf(c, exp2f(sp.k * __log2f(x)), s);
+#ifdef __CUDA_ARCH__
+                if (c && x > 0.0f) s = fmaf((float)c, exp2f(sp.k * __log2f(x)), s);
+#else
+                if (c && x > 0.0f) s = fmaf((float)c, exp2f(sp.k * log2f(x)), s);
+#endif
             }
             if (s >= thr) ulo = um; else uhi = um;
         }
-        return ((float)(h.top - J) + ulo) * sp.w;
+        tau_h = ((float)(h.top - J) + ulo) * sp.w;
     }
+    return tau_h - 4.0f * 1.1920929e-7f * fmaxf(1.0f, fabsf(tau_h));
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -74,6 +74,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
     uint32_t* cand = reinterpret_cast<uint32_t*>(Tk + 260);        // [cwords]
     uint32_t* next = cand + cwords;                                // [cwords]
     uint32_t* mrow = next + cwords;                                // [mrows][nw]
+    uint32_t* live_all = mrow + mrows * a.nw;                      // [128][kLiveStride]
     __shared__ TileStats st;
 
     const int tid = threadIdx.x;
@@ -104,7 +105,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
 
     // ---- sweep 1: dense scores, running max, histogram, candidate blocks ----
     HistRow h;
-    hist_init(h);
+    hist_init(h, live_all, tid);
     Stash sh;
     sh.n = 0;
     sh.overflow = false;
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
         }
         bool any = false;
         if (sp.init_mode == 0) {
-            hist_raise(h, amax, sp, hist, tid);
+            hist_raise(h, amax, sp.cbin, sp.inv_cz, sp.bins);
         } else if (amax > h.m_raw) {
             h.m_raw = amax;
             h.thr_raw = amax - sp.inv_cz;
@@ -131,7 +132,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
         for (int jj = 0; jj < mb; ++jj)
             if (sc[jj] > h.thr_raw) {
                 any = true;
-                if (sp.init_mode == 0) hist_add(h, sc[jj], sp, hist, tid);
+                if (sp.init_mode == 0) hist_add(h, sc[jj], sp.cbin, sp.bins, hist, tid);
                 stash_add(sh, sc[jj], h.thr_raw, stash, tid);
             }
         if (any) atomicOr(&cand[J >> 5], 1u << (J & 31));
@@ -304,7 +305,7 @@ cudaError_t launch_t(const FwdArgs& a, cudaStream_t stream) {
     const int mrows = kTileRows / a.mb;
     const size_t uni_words = (size_t)max(256 * kTileRows, 2 * D * kTileRows);
     const size_t bytes = (size_t)2 * kKeyBlk * D * 4 + uni_words * 4 + 260 * 4 +
-                         (size_t)(2 * cwords + mrows * a.nw) * 4;
+                         (size_t)(2 * cwords + mrows * a.nw) * 4 + (size_t)kTileRows * kLiveStride * 4;
     auto kern = fwd_simt_kernel<T, D, KIND>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;

@@ -31,8 +31,9 @@ constexpr int BM = 128;           // query rows per tile
 constexpr int BN = 64;            // keys per block (= mask block)
 constexpr int NVS = 2;            // V ring stages
 constexpr int kThreads = 192;
-constexpr uint32_t kHistBytes = 256u * BM * 2u + kStashCap * BM * 4u;  // histogram + stash (128 KB), reused
-                                                                       // for V / P / U after the dense sweep
+constexpr uint32_t kRowBufStride = 68;  // floats per row of the rare-path buffer (16-byte aligned, no conflicts)
+// dense sweep: histogram (u16, 64 KB) + stash (32 KB) + rare-path row buffer (34 KB); the V ring after it
+constexpr uint32_t kHistBytes = 256u * BM * 2u + kStashCap * BM * 4u + BM * kRowBufStride * 4u;
 
 template <int D>
 struct Cfg {
@@ -42,19 +43,18 @@ struct Cfg {
     static constexpr uint32_t kPBytes = BM * BN * 2;       // 16 KB
     static constexpr uint32_t offQ = 0;
     static constexpr uint32_t offK = offQ + kQBytes;
-    static constexpr int NPB = (D == 64) ? 2 : 1;          // P / U buffer sets
-    static constexpr uint32_t offU = offK + NKS * kKBytes;  // union region
-    static constexpr uint32_t offV = offU;                  // V ring inside the union
-    static constexpr uint32_t offP = offV + NVS * kKBytes;  // P buffers [NPB] (bf16 high part)
-    static constexpr uint32_t offPL = offP + NPB * kPBytes; // P buffers [NPB] (bf16 low part)
-    static constexpr uint32_t offUU = offPL + NPB * kPBytes;  // U buffers [NPB] (bf16 high part)
-    static constexpr uint32_t offUL = offUU + NPB * kPBytes;  // U buffers [NPB] (bf16 low part)
-    static constexpr uint32_t kUnion =
-        (kHistBytes > NVS * kKBytes + 4 * NPB * kPBytes) ? kHistBytes : NVS * kKBytes + 4 * NPB * kPBytes;
-    static constexpr uint32_t offSmall = offU + kUnion;
+    static constexpr int NPB = (D == 64) ? 2 : 1;          // P / U buffer sets in TMEM
+    static constexpr uint32_t offU = offK + NKS * kKBytes;  // union region: histogram + stash, then V ring
+    static constexpr uint32_t offV = offU;
+    static_assert(NVS * kKBytes <= kHistBytes, "V ring must fit the union region");
+    static constexpr uint32_t offSmall = offU + kHistBytes;
     static constexpr uint32_t tmemCols = 512;
     static constexpr uint32_t colO = 128;
     static constexpr uint32_t colOb = 128 + D;
+    // P / U operands of the P V and U V MMAs live in TMEM (A operand from tensor memory): per buffer set
+    // 4 tiles of 128 lanes x 32 columns (64 bf16 per row): P high, P low, U high, U low.
+    static constexpr uint32_t colP = 128 + 2 * D;
+    static_assert(colP + NPB * 128 <= tmemCols, "TMEM budget");
 };
 
 struct Small {
@@ -95,6 +95,41 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
+// Out-of-line path of the dense sweep, taken when a row's stash is nearly full: drop the entries that
+// fell below the threshold; if the stash stays more than half full, the row switches to streaming its
+// histogram (its stash is binned now) and is marked overflowed. Returns the new stash count, or -1.
+static __device__ __noinline__ int stash_room(int n, HistRow& h, float* stash, uint16_t* hist, int r, float m_run,
+                                              float thr, float cbin, int bins, int init_mode) {
+    int j = 0;
+    for (int i = 0; i < n; ++i) {
+        const float v = stash[i * kTileRows + r];
+        if (v > thr) stash[(j++) * kTileRows + r] = v;
+    }
+    if (j <= kStashCap / 2) return j;
+    if (init_mode == 0) {
+        Stash st;
+        st.n = j;
+        st.overflow = false;
+        hist_from_stash(h, st, stash, m_run, thr, cbin, bins, hist, r);
+    }
+    return -1;
+}
+
+// Streaming path for a row whose stash overflowed: bin this block's entries above the threshold
+// (rolled loop over the row's scores, staged in shared memory).
+static __device__ __noinline__ void stream_block(HistRow& h, const float* rb, uint32_t gflag, float thr, float cbin,
+                                                 int bins, int init_mode, uint16_t* hist, int r) {
+    if (init_mode != 0) return;
+    while (gflag) {
+        const int g = __ffs(gflag) - 1;
+        gflag &= gflag - 1;
+        for (int e = 0; e < 8; ++e) {
+            const float v = rb[8 * g + e];
+            if (v > thr) hist_add(h, v, cbin, bins, hist, r);
+        }
+    }
+}
+
 __device__ __forceinline__ bool block_full(int J, int n, int causal, int row0) {
     const int last = J * BN + BN - 1;
     return last < n && (!causal || last <= row0);
@@ -114,8 +149,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* plan_bits = reinterpret_cast<uint32_t*>(&sm + 1);  // [2][W]
     uint32_t* next = plan_bits + 2 * W;                          // [W]
     uint32_t* mrow = next + W;                                   // [2][W]
-    uint16_t* hist = reinterpret_cast<uint16_t*>(smem + C::offU);                 // [256][128] u16, 64 KB
-    float* stash = reinterpret_cast<float*>(smem + C::offU + 256 * BM * 2);        // [kStashCap][128], 64 KB
+    uint16_t* hist = reinterpret_cast<uint16_t*>(smem + C::offU);                 // [256][128] u16
+    float* stash = reinterpret_cast<float*>(smem + C::offU + 256 * BM * 2);        // [kStashCap][128]
+    float* rowbuf = stash + kStashCap * BM;                                        // [128][kRowBufStride]
+    uint32_t* live_all = mrow + 2 * W;                                             // [128][kLiveStride]
 
     const SolveParams sp = a.sp;
     const int tid = threadIdx.x;
@@ -154,10 +191,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sQ = smem_u32(smem + C::offQ);
     const uint32_t sK0 = smem_u32(smem + C::offK);
     const uint32_t sV0 = smem_u32(smem + C::offV);
-    const uint32_t sP0 = smem_u32(smem + C::offP);
-    const uint32_t sPL0 = smem_u32(smem + C::offPL);
-    const uint32_t sU0 = smem_u32(smem + C::offUU);
-    const uint32_t sUL0 = smem_u32(smem + C::offUL);
 
     if (warp == 5) {
         // ------------------------------------------------------------------ TMA issue
@@ -171,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t lc = 0, vc = 0;
             bool ok = true;
             for (int sw = 0; ok; ++sw) {
-                if (!(ok = wait_bounded(&sm.ctrl, sw & 1, abort_flag, a.status))) break;
+                if (!(ok = wait_bounded(&sm.ctrl, sw & 1, abort_flag, a.status, true))) break;
                 const int kind = sm.plan_kind[sw & 1];
                 if (kind == kSweepDone) break;
                 const uint32_t* bits_p = plan_bits + (sw & 1) * W;
@@ -181,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int J = wd * 32 + __ffs(bits) - 1;
                         bits &= bits - 1;
                         const uint32_t ks = lc % C::NKS;
-                        if (!(ok = wait_bounded(&sm.k_empty[ks], ((lc / C::NKS) & 1) ^ 1, abort_flag, a.status))) break;
+                        if (!(ok = wait_bounded(&sm.k_empty[ks], ((lc / C::NKS) & 1) ^ 1, abort_flag, a.status, true))) break;
                         mbar_arrive_expect_tx(&sm.k_full[ks], C::kKBytes);
                         for (int c = 0; c < D / 64; ++c)
                             tma_load_3d(smem + C::offK + ks * C::kKBytes + c * (BN * 128), &tmK, &sm.k_full[ks],
@@ -189,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ++lc;
                         if (kind == kSweepPV) {
                             const uint32_t vs = vc % NVS;
-                            if (!(ok = wait_bounded(&sm.v_empty[vs], ((vc / NVS) & 1) ^ 1, abort_flag, a.status))) break;
+                            if (!(ok = wait_bounded(&sm.v_empty[vs], ((vc / NVS) & 1) ^ 1, abort_flag, a.status, true))) break;
                             mbar_arrive_expect_tx(&sm.v_full[vs], C::kKBytes);
                             for (int c = 0; c < D / 64; ++c)
                                 tma_load_3d(smem + C::offV + vs * C::kKBytes + c * (BN * 128), &tmV,
@@ -214,12 +247,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
             constexpr uint32_t idPV = idesc_bf16_f32(BM, D, false, true);
             uint32_t lc = 0, vc = 0, sc = 0, pc = 0;
-            bool ok = wait_bounded(&sm.q_full, 0, abort_flag, a.status);
+            bool ok = wait_bounded(&sm.q_full, 0, abort_flag, a.status, true);
             tc_fence_after();
             auto issue_S = [&](uint32_t ks) -> bool {
                 const uint32_t sb = sc & 1;
-                if (!wait_bounded(&sm.k_full[ks], (lc / C::NKS) & 1, abort_flag, a.status)) return false;
-                if (!wait_bounded(&sm.s_empty[sb], ((sc >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&sm.k_full[ks], (lc / C::NKS) & 1, abort_flag, a.status, true)) return false;
+                if (!wait_bounded(&sm.s_empty[sb], ((sc >> 1) & 1) ^ 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t kbase = sK0 + ks * C::kKBytes;
 #pragma unroll
@@ -238,24 +271,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto issue_PV = [&](bool first) -> bool {
                 const uint32_t pb = pc % C::NPB;
                 const uint32_t vs = vc % NVS;
-                if (!wait_bounded(&sm.p_full[pb], (pc / C::NPB) & 1, abort_flag, a.status)) return false;
-                if (!wait_bounded(&sm.v_full[vs], (vc / NVS) & 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&sm.p_full[pb], (pc / C::NPB) & 1, abort_flag, a.status, true)) return false;
+                if (!wait_bounded(&sm.v_full[vs], (vc / NVS) & 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t vbase = sV0 + vs * C::kKBytes;
+                const uint32_t tp = tmem + C::colP + pb * 128;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
                     const uint64_t dv = sdesc_sw128(vbase + kk * 2048, BN * 128, 1024);
-                    const uint64_t dp = sdesc_sw128(sP0 + pb * C::kPBytes + kk * 32, 16, 1024);
-                    const uint64_t dpl = sdesc_sw128(sPL0 + pb * C::kPBytes + kk * 32, 16, 1024);
-                    const uint64_t du = sdesc_sw128(sU0 + pb * C::kPBytes + kk * 32, 16, 1024);
-                    const uint64_t dul = sdesc_sw128(sUL0 + pb * C::kPBytes + kk * 32, 16, 1024);
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
                     // P = P_hi + P_lo and U = U_hi + U_lo (two bf16 terms each) keep P V and U V accurate
-                    // to ~16 mantissa bits
-                    mma_bf16_ss(tmem + C::colO, dp, dv, idPV, acc);
-                    mma_bf16_ss(tmem + C::colO, dpl, dv, idPV, 1u);
-                    mma_bf16_ss(tmem + C::colOb, du, dv, idPV, acc);
-                    mma_bf16_ss(tmem + C::colOb, dul, dv, idPV, 1u);
+                    // to ~16 mantissa bits; each K step of 16 keys is 8 TMEM columns of the A tile
+                    mma_bf16_ts(tmem + C::colO, tp + 0 + kk * 8, dv, idPV, acc);
+                    mma_bf16_ts(tmem + C::colO, tp + 32 + kk * 8, dv, idPV, 1u);
+                    mma_bf16_ts(tmem + C::colOb, tp + 64 + kk * 8, dv, idPV, acc);
+                    mma_bf16_ts(tmem + C::colOb, tp + 96 + kk * 8, dv, idPV, 1u);
                 }
                 mma_commit(&sm.p_empty[pb]);
                 mma_commit(&sm.v_empty[vs]);
@@ -264,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             for (int sw = 0; ok; ++sw) {
-                if (!(ok = wait_bounded(&sm.ctrl, sw & 1, abort_flag, a.status))) break;
+                if (!(ok = wait_bounded(&sm.ctrl, sw & 1, abort_flag, a.status, true))) break;
                 const int kind = sm.plan_kind[sw & 1];
                 if (kind == kSweepDone) break;
                 const uint32_t* bits_p = plan_bits + (sw & 1) * W;
@@ -373,39 +403,82 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // ---- sweep 0: dense ----
         HistRow h;
-        hist_init(h);
+        hist_init(h, live_all, r);
         Stash sh;
         sh.n = 0;
         sh.overflow = false;
+        // Candidates (z > running max - 1) go to the stash; the histogram is built from the stash when
+        // the sweep ends (one binning per candidate instead of one window update per block). Rows whose
+        // stash overflows stream their histogram from then on.
+        float m_run = -INFINITY, thr = INFINITY;
+        int nst = 0;           // stash entries
+        bool ovf = false;      // stash overflowed: streaming histogram
         for (int J = 0; J < nblk && ok; ++J) {
             if (!(ok = load_S())) break;
             mask_S(J);
             const float amax = group_max();
-            if (sp.init_mode == 0) {
-                hist_raise(h, amax, sp, hist, r);
-            } else if (amax > h.m_raw) {
-                h.m_raw = amax; h.thr_raw = amax - sp.inv_cz; h.any = true;
+            if (amax > m_run) {
+                m_run = amax;
+                thr = amax - sp.inv_cz;
+                if (ovf && sp.init_mode == 0) hist_raise(h, amax, sp.cbin, sp.inv_cz, sp.bins);
             }
-            const bool any = amax > h.thr_raw;
+            const bool any = amax > thr;
             if (any) {
+                if (!ovf) {
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    if (gm[g] > h.thr_raw) {
+                    for (int g = 0; g < 8; ++g) {
+                        if (gm[g] > thr) {
+                            if (nst > kStashCap - 8) {
+                                nst = stash_room(nst, h, stash, hist, r, m_run, thr, sp.cbin, sp.bins, sp.init_mode);
+                                if (nst < 0) { ovf = true; nst = 0; }
+                            }
+                            if (!ovf) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float v = vbuf[8 * g + e];
-                            if (v > h.thr_raw) {
-                                if (sp.init_mode == 0) hist_add(h, v, sp, hist, r);
-                                stash_add(sh, v, h.thr_raw, stash, r);
+                                for (int e = 0; e < 8; ++e) {
+                                    const float v = vbuf[8 * g + e];
+                                    if (v > thr) {
+                                        stash[nst * BM + r] = v;
+                                        ++nst;
+                                    }
+                                }
+                            } else {
+                                // switched to streaming in this block: bin the rest of it
+                                uint32_t gflag = 0u;
+#pragma unroll
+                                for (int g2 = 0; g2 < 8; ++g2) gflag |= (g2 >= g && gm[g2] > thr ? 1u : 0u) << g2;
+                                float* rb = rowbuf + r * kRowBufStride;
+#pragma unroll
+                                for (int c = 0; c < BN; c += 4)
+                                    *reinterpret_cast<float4*>(rb + c) =
+                                        make_float4(vbuf[c], vbuf[c + 1], vbuf[c + 2], vbuf[c + 3]);
+                                stream_block(h, rb, gflag, thr, sp.cbin, sp.bins, sp.init_mode, hist, r);
+                                break;
                             }
                         }
                     }
+                } else {
+                    uint32_t gflag = 0u;
+#pragma unroll
+                    for (int g = 0; g < 8; ++g) gflag |= (gm[g] > thr ? 1u : 0u) << g;
+                    float* rb = rowbuf + r * kRowBufStride;
+#pragma unroll
+                    for (int c = 0; c < BN; c += 4)
+                        *reinterpret_cast<float4*>(rb + c) = make_float4(vbuf[c], vbuf[c + 1], vbuf[c + 2], vbuf[c + 3]);
+                    stream_block(h, rb, gflag, thr, sp.cbin, sp.bins, sp.init_mode, hist, r);
                 }
             }
             const uint32_t ball = __ballot_sync(0xffffffffu, any);
             if (lane == 0 && ball) atomicOr(&next[J >> 5], 1u << (J & 31));
         }
         ok = !bar_or_compute(!ok || *abort_flag != 0);
+        sh.n = nst;
+        sh.overflow = ovf;
+        if (!ovf) {
+            if (sp.init_mode == 0) hist_from_stash(h, sh, stash, m_run, thr, sp.cbin, sp.bins, hist, r);
+            h.m_raw = m_run;
+            h.thr_raw = thr;
+            h.any = m_run > -INFINITY;
+        }
 
         const float m = sp.cz * h.m_raw;
         float tau_h = m - 1.0f;
@@ -501,59 +574,63 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = __all_sync(0xffffffffu,
                                     wait_bounded(&sm.p_empty[pb], ((pc / C::NPB) & 1) ^ 1, abort_flag, a.status));
                     if (!ok) break;
-                    const uint32_t pbase = sP0 + pb * C::kPBytes;
-                    const uint32_t plbase = sPL0 + pb * C::kPBytes;
-                    const uint32_t ubase = sU0 + pb * C::kPBytes;
-                    const uint32_t ulbase = sUL0 + pb * C::kPBytes;
+                    const uint32_t tp = lane_base + C::colP + pb * 128;
 #pragma unroll
-                    for (int g = 0; g < 8; ++g) {
-                        uint32_t ph[4] = {0u, 0u, 0u, 0u}, pl[4] = {0u, 0u, 0u, 0u}, uu[4] = {0u, 0u, 0u, 0u};
-                        uint32_t ul[4] = {0u, 0u, 0u, 0u};
-                        if (sp.cz * gm[g] - t > 0.f) {
+                    for (int gp = 0; gp < 4; ++gp) {
+                        // two groups of 8 keys = 8 TMEM columns of each of the four A tiles
+                        uint32_t ph[8], pl[8], uh[8], ul[8];
 #pragma unroll
-                            for (int e = 0; e < 8; e += 2) {
-                                float pv2[2], uv2[2];
+                        for (int q8 = 0; q8 < 2; ++q8) {
+                            const int g = 2 * gp + q8;
+                            if (sp.cz * gm[g] - t > 0.f) {
 #pragma unroll
-                                for (int q = 0; q < 2; ++q) {
-                                    const float x = sp.cz * vbuf[8 * g + e + q] - t;
-                                    float p, u;
-                                    if constexpr (KIND == kAlpha15) {
-                                        u = fmaxf(x, 0.f);
-                                        p = u * u;
-                                        F2 += x > 0.f ? 1.f : 0.f;
-                                    } else if constexpr (KIND == kAlpha2) {
-                                        p = fmaxf(x, 0.f);
-                                        u = x > 0.f ? 1.f : 0.f;
-                                    } else {
-                                        const bool pos = x > 0.f;
-                                        const float xs = pos ? x : 1.f;
-                                        const float uu1 = exp2f((sp.k - 1.f) * __log2f(xs));
-                                        u = pos ? uu1 : 0.f;
-                                        p = u * xs;
-                                        F2 += pos ? __fdividef(uu1, xs) : 0.f;
+                                for (int e = 0; e < 8; e += 2) {
+                                    float pv2[2], uv2[2];
+#pragma unroll
+                                    for (int q = 0; q < 2; ++q) {
+                                        const float x = sp.cz * vbuf[8 * g + e + q] - t;
+                                        float p, u;
+                                        if constexpr (KIND == kAlpha15) {
+                                            u = fmaxf(x, 0.f);
+                                            p = u * u;
+                                            F2 += x > 0.f ? 1.f : 0.f;
+                                        } else if constexpr (KIND == kAlpha2) {
+                                            p = fmaxf(x, 0.f);
+                                            u = x > 0.f ? 1.f : 0.f;
+                                        } else {
+                                            const bool pos = x > 0.f;
+                                            const float xs = pos ? x : 1.f;
+                                            const float uu1 = exp2f((sp.k - 1.f) * __log2f(xs));
+                                            u = pos ? uu1 : 0.f;
+                                            p = u * xs;
+                                            F2 += pos ? __fdividef(uu1, xs) : 0.f;
+                                        }
+                                        Sp += p;
+                                        Su += u;
+                                        pv2[q] = p;
+                                        uv2[q] = u;
                                     }
-                                    Sp += p;
-                                    Su += u;
-                                    pv2[q] = p;
-                                    uv2[q] = u;
+                                    const int w = q8 * 4 + e / 2;
+                                    const __nv_bfloat162 hi = __floats2bfloat162_rn(pv2[0], pv2[1]);
+                                    const float2 hf = __bfloat1622float2(hi);
+                                    ph[w] = *reinterpret_cast<const uint32_t*>(&hi);
+                                    pl[w] = pack_bf16x2(pv2[0] - hf.x, pv2[1] - hf.y);
+                                    const __nv_bfloat162 uh2 = __floats2bfloat162_rn(uv2[0], uv2[1]);
+                                    const float2 uf = __bfloat1622float2(uh2);
+                                    uh[w] = *reinterpret_cast<const uint32_t*>(&uh2);
+                                    ul[w] = pack_bf16x2(uv2[0] - uf.x, uv2[1] - uf.y);
                                 }
-                                const __nv_bfloat162 hi = __floats2bfloat162_rn(pv2[0], pv2[1]);
-                                const float2 hf = __bfloat1622float2(hi);
-                                ph[e / 2] = *reinterpret_cast<const uint32_t*>(&hi);
-                                pl[e / 2] = pack_bf16x2(pv2[0] - hf.x, pv2[1] - hf.y);
-                                const __nv_bfloat162 uh = __floats2bfloat162_rn(uv2[0], uv2[1]);
-                                const float2 uf = __bfloat1622float2(uh);
-                                uu[e / 2] = *reinterpret_cast<const uint32_t*>(&uh);
-                                ul[e / 2] = pack_bf16x2(uv2[0] - uf.x, uv2[1] - uf.y);
+                            } else {
+#pragma unroll
+                                for (int w = q8 * 4; w < q8 * 4 + 4; ++w) ph[w] = pl[w] = uh[w] = ul[w] = 0u;
                             }
                         }
-                        const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)g);
-                        st_shared_v4(pbase + off, ph[0], ph[1], ph[2], ph[3]);
-                        st_shared_v4(plbase + off, pl[0], pl[1], pl[2], pl[3]);
-                        st_shared_v4(ubase + off, uu[0], uu[1], uu[2], uu[3]);
-                        st_shared_v4(ulbase + off, ul[0], ul[1], ul[2], ul[3]);
+                        tmem_st8(tp + 0 + gp * 8, ph);
+                        tmem_st8(tp + 32 + gp * 8, pl);
+                        tmem_st8(tp + 64 + gp * 8, uh);
+                        tmem_st8(tp + 96 + gp * 8, ul);
                     }
-                    fence_proxy_async_smem();
+                    tmem_st_wait();
                     mbar_arrive(&sm.p_full[pb]);
                     ++pc;
                     const uint32_t kb = __ballot_sync(0xffffffffu, keep);
@@ -711,7 +788,7 @@ static cudaError_t launch_fwd_tc_t(const FwdArgs& a, cudaStream_t stream) {
     if ((e = make_tmap_bf16(&tq, a.Q, a.B * a.H, a.n, D, BM)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16(&tk, a.K, a.B * a.H, a.n, D, BN)) != cudaSuccess) return e;
     if ((e = make_tmap_bf16(&tv, a.V, a.B * a.H, a.n, D, BN)) != cudaSuccess) return e;
-    const size_t bytes = 1024 + C::offSmall + sizeof(Small) + (size_t)5 * a.nw * 4;
+    const size_t bytes = 1024 + C::offSmall + sizeof(Small) + (size_t)5 * a.nw * 4 + (size_t)BM * kLiveStride * 4;
     if (bytes > 232448) return cudaErrorInvalidConfiguration;
     auto kern = fwd_tc_kernel<D, KIND>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
@@ -722,7 +799,7 @@ static cudaError_t launch_fwd_tc_t(const FwdArgs& a, cudaStream_t stream) {
 }
 
 size_t fwd_tc_smem_bytes(int d, int nw) {
-    const size_t small = sizeof(Small) + (size_t)5 * nw * 4;
+    const size_t small = sizeof(Small) + (size_t)5 * nw * 4 + (size_t)BM * kLiveStride * 4;
     return 1024 + (d == 64 ? Cfg<64>::offSmall : Cfg<128>::offSmall) + small;
 }
 

@@ -56,7 +56,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
         "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -111,7 +110,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int J = 0;
             for (; J < nblk && ok; ++J) {
                 const int st = J % NST;
-                if (!(ok = wait_bounded(&bb.kv_empty[st], ((J / NST) & 1) ^ 1, abort_flag, a.status))) break;
+                if (!(ok = wait_bounded(&bb.kv_empty[st], ((J / NST) & 1) ^ 1, abort_flag, a.status, true))) break;
                 unsigned char* base = smem + C::offSt + st * C::kStage;
                 mbar_arrive_expect_tx(&bb.kv_full[st], C::kStage);
                 for (int c = 0; c < D / 64; ++c) {
@@ -128,12 +127,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idS = idesc_bf16_f32(BM, BN, false, false);
             constexpr uint32_t idPV = idesc_bf16_f32(BM, D, false, true);
-            bool ok = wait_bounded(&bb.q_full, 0, abort_flag, a.status);
+            bool ok = wait_bounded(&bb.q_full, 0, abort_flag, a.status, true);
             tc_fence_after();
             auto issue_S = [&](int J) -> bool {
                 const int st = J % NST, sb = J & 1;
-                if (!wait_bounded(&bb.kv_full[st], (J / NST) & 1, abort_flag, a.status)) return false;
-                if (!wait_bounded(&bb.s_empty[sb], ((J >> 1) & 1) ^ 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&bb.kv_full[st], (J / NST) & 1, abort_flag, a.status, true)) return false;
+                if (!wait_bounded(&bb.s_empty[sb], ((J >> 1) & 1) ^ 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t kb = sSt + st * C::kStage;
 #pragma unroll
@@ -147,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto issue_PV = [&](int J) -> bool {
                 const int st = J % NST, pb = J & 1;
-                if (!wait_bounded(&bb.p_full[pb], (J >> 1) & 1, abort_flag, a.status)) return false;
+                if (!wait_bounded(&bb.p_full[pb], (J >> 1) & 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t vb = sSt + st * C::kStage + C::kBlk;
 #pragma unroll
