@@ -80,17 +80,16 @@ __device__ __forceinline__ void pointwise(float s, float stat, float cz, float k
     }
 }
 
-// Pack 8 values into one 16-byte chunk of bf16 (high part) and, with SPLIT, the low part.
+// Two values as a bf16 pair (high part) and, with SPLIT, the bf16 pair of the remainders (low part).
 template <bool SPLIT>
-__device__ __forceinline__ void pack8(const float* v, uint32_t* hi, uint32_t* lo) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-        hi[i] = *reinterpret_cast<const uint32_t*>(&h);
-        if constexpr (SPLIT) {
-            const float2 hf = __bfloat1622float2(h);
-            lo[i] = pack_bf16x2(v[2 * i] - hf.x, v[2 * i + 1] - hf.y);
-        }
+__device__ __forceinline__ void split2(const float* v, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v[0], v[1]);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    if constexpr (SPLIT) {
+        const float2 hf = __bfloat1622float2(h);
+        lo = pack_bf16x2(v[0] - hf.x, v[1] - hf.y);
+    } else {
+        lo = 0u;
     }
 }
 
@@ -143,17 +142,20 @@ struct CfgKV {
     static constexpr uint32_t kTile = TM * D * 2;   // K or V tile, 16 / 32 KB
     static constexpr uint32_t kBlk = TB * D * 2;    // Q_I or dO_I block, 8 / 16 KB
     static constexpr uint32_t kStage = 2 * kBlk + 1024;  // Q_I, dO_I, stat[64], delta[64] (+ pad)
-    static constexpr uint32_t kPT = TM * TB * 2;    // P^T or dS^T tile (bf16), 16 KB
     static constexpr uint32_t offK = 0;
     static constexpr uint32_t offV = offK + kTile;
     static constexpr uint32_t offSt = offV + kTile;               // 2 stages
-    static constexpr uint32_t offP = offSt + 2 * kStage;          // P^T hi, P^T lo, dS^T hi, dS^T lo
-    static constexpr uint32_t offBar = offP + 4 * kPT;
-    static constexpr uint32_t colS = 0;    // S^T double buffer: [0,64) [64,128)
-    static constexpr uint32_t colDP = 128; // dP^T double buffer: [128,192) [192,256)
-    static constexpr uint32_t colDV = 256;
-    static constexpr uint32_t colDK = 256 + D;
+    static constexpr uint32_t offBar = offSt + 2 * kStage;
+    // TMEM: S^T and dP^T (double-buffered at d = 64), dV, dK, and the A tiles of the gradient MMAs
+    // (P^T hi, P^T lo, dS^T hi, dS^T lo: 4 x 32 columns, bf16 pairs), read by tcgen05.mma from TMEM.
+    static constexpr int NSB = (D == 64) ? 2 : 1;
+    static constexpr uint32_t colS = 0;
+    static constexpr uint32_t colDP = NSB * TB;
+    static constexpr uint32_t colDV = 2 * NSB * TB;
+    static constexpr uint32_t colDK = colDV + D;
+    static constexpr uint32_t colA = colDK + D;
     static constexpr uint32_t tmemCols = 512;
+    static_assert(colA + 128 <= tmemCols, "TMEM budget");
 };
 
 struct BarsKV {
@@ -228,7 +230,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sK = smem_u32(smem + C::offK);
     const uint32_t sV = smem_u32(smem + C::offV);
     const uint32_t sSt = smem_u32(smem + C::offSt);
-    const uint32_t sP = smem_u32(smem + C::offP);
 
     if (warp == 5) {
         if (lane == 0) {
@@ -271,9 +272,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             uint32_t i = 0;
             auto issue_S = [&](uint32_t idx) -> bool {
-                const uint32_t st = idx & 1, sb = idx & 1;
+                const uint32_t st = idx & 1, sb = idx % C::NSB;
                 if (!wait_bounded(&bb.q_full[st], (idx >> 1) & 1, abort_flag, a.status, true)) return false;
-                if (!wait_bounded(&bb.s_empty[sb], ((idx >> 1) & 1) ^ 1, abort_flag, a.status, true)) return false;
+                if (!wait_bounded(&bb.s_empty[sb], ((idx / C::NSB) & 1) ^ 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t qb = sSt + st * C::kStage, ob = qb + C::kBlk;
 #pragma unroll
@@ -298,15 +299,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < TB / 16; ++kk) {
                     const uint64_t dob = sdesc_sw128(ob + kk * 2048, TB * 128, 1024);
                     const uint64_t dqb = sdesc_sw128(qb + kk * 2048, TB * 128, 1024);
-                    const uint64_t pth = sdesc_sw128(sP + 0 * C::kPT + kk * 32, 16, 1024);
-                    const uint64_t ptl = sdesc_sw128(sP + 1 * C::kPT + kk * 32, 16, 1024);
-                    const uint64_t dsh = sdesc_sw128(sP + 2 * C::kPT + kk * 32, 16, 1024);
-                    const uint64_t dsl = sdesc_sw128(sP + 3 * C::kPT + kk * 32, 16, 1024);
+                    const uint32_t ta = tmem + C::colA + kk * 8;  // 16 query rows = 8 TMEM columns
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-                    mma_bf16_ss(tmem + C::colDV, pth, dob, idG, acc);
-                    if constexpr (SPLIT) mma_bf16_ss(tmem + C::colDV, ptl, dob, idG, 1u);
-                    mma_bf16_ss(tmem + C::colDK, dsh, dqb, idG, acc);
-                    if constexpr (SPLIT) mma_bf16_ss(tmem + C::colDK, dsl, dqb, idG, 1u);
+                    mma_bf16_ts(tmem + C::colDV, ta + 0, dob, idG, acc);
+                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDV, ta + 32, dob, idG, 1u);
+                    mma_bf16_ts(tmem + C::colDK, ta + 64, dqb, idG, acc);
+                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDK, ta + 96, dqb, idG, 1u);
                 }
                 mma_commit(&bb.ds_empty);
                 mma_commit(&bb.q_empty[st]);
@@ -337,8 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (bits) {
                 const int I = w * 32 + __ffs(bits) - 1;
                 bits &= bits - 1;
-                const uint32_t sb = i & 1, st = i & 1;
-                ok = __all_sync(0xffffffffu, wait_bounded(&bb.s_full[sb], (i >> 1) & 1, abort_flag, a.status));
+                const uint32_t sb = i % C::NSB, st = i & 1;
+                ok = __all_sync(0xffffffffu, wait_bounded(&bb.s_full[sb], (i / C::NSB) & 1, abort_flag, a.status));
                 if (!ok) break;
                 tc_fence_after();
                 __syncwarp();
@@ -356,31 +354,59 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float* dl = stat + 64;
                 const int q0 = I * TB;
                 const bool full = kvalid && (q0 + TB <= a.n) && (!a.causal || q0 >= k0 + TM - 1);
-                // P^T and dS^T rows for this key against the 64 query rows of block I
-                float pv[TB], dsv[TB];
-#pragma unroll
-                for (int c = 0; c < TB; ++c) {
-                    const int qi = q0 + c;
-                    const bool okc = full || (kvalid && qi < a.n && (!a.causal || qi >= key));
-                    float p, u;
-                    pointwise<MODE>(sv[c], stat[c], a.cz, a.k, okc, p, u);
-                    pv[c] = p;
-                    dsv[c] = u * (dpv[c] - dl[c]);
-                }
+                // the A tiles of the previous block's gradient MMAs must have been read
                 ok = __all_sync(0xffffffffu, wait_bounded(&bb.ds_empty, (i & 1) ^ 1, abort_flag, a.status));
                 if (!ok) break;
+                const uint32_t ta = lane_base + C::colA;
+                // P^T and dS^T rows for this key against the 64 query rows of block I, 16 columns at a time
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    uint32_t ph[4], pl[4], dh[4], dlo[4];
-                    pack8<SPLIT>(pv + 8 * g, ph, pl);
-                    pack8<SPLIT>(dsv + 8 * g, dh, dlo);
-                    const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)g);
-                    st_shared_v4(sP + 0 * C::kPT + off, ph[0], ph[1], ph[2], ph[3]);
-                    if constexpr (SPLIT) st_shared_v4(sP + 1 * C::kPT + off, pl[0], pl[1], pl[2], pl[3]);
-                    st_shared_v4(sP + 2 * C::kPT + off, dh[0], dh[1], dh[2], dh[3]);
-                    if constexpr (SPLIT) st_shared_v4(sP + 3 * C::kPT + off, dlo[0], dlo[1], dlo[2], dlo[3]);
+                for (int gp = 0; gp < 4; ++gp) {
+                    uint32_t ph[8], pl[8], dh[8], dlo[8];
+                    float st16[16], dl16[16];
+#pragma unroll
+                    for (int i4 = 0; i4 < 4; ++i4) {  // broadcast loads of the 16 columns' statistics
+                        const float4 a4 = *reinterpret_cast<const float4*>(stat + 16 * gp + 4 * i4);
+                        const float4 b4 = *reinterpret_cast<const float4*>(dl + 16 * gp + 4 * i4);
+                        st16[4 * i4] = a4.x; st16[4 * i4 + 1] = a4.y; st16[4 * i4 + 2] = a4.z; st16[4 * i4 + 3] = a4.w;
+                        dl16[4 * i4] = b4.x; dl16[4 * i4 + 1] = b4.y; dl16[4 * i4 + 2] = b4.z; dl16[4 * i4 + 3] = b4.w;
+                    }
+                    // entmax: 16 columns with no positive z - tau give P = dS = 0 (the usual case)
+                    bool anyx = (MODE == kModeSoftmax);
+                    if constexpr (MODE != kModeSoftmax) {
+                        float xm = -1.f;
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) xm = fmaxf(xm, fmaf(sv[16 * gp + e], a.cz, -st16[e]));
+                        anyx = xm > 0.f;
+                    }
+                    if (anyx) {
+#pragma unroll
+                    for (int q2 = 0; q2 < 8; ++q2) {
+                        float pp[2], dd[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int cc = 2 * q2 + e;
+                            const int c = 16 * gp + cc;
+                            const int qi = q0 + c;
+                            const bool okc = full || (kvalid && qi < a.n && (!a.causal || qi >= key));
+                            float p, u;
+                            pointwise<MODE>(sv[c], st16[cc], a.cz, a.k, okc, p, u);
+                            pp[e] = p;
+                            dd[e] = u * (dpv[c] - dl16[cc]);
+                        }
+                        split2<SPLIT>(pp, ph[q2], pl[q2]);
+                        split2<SPLIT>(dd, dh[q2], dlo[q2]);
+                    }
+                    } else {
+#pragma unroll
+                        for (int q2 = 0; q2 < 8; ++q2) ph[q2] = pl[q2] = dh[q2] = dlo[q2] = 0u;
+                    }
+                    tmem_st8(ta + 0 + gp * 8, ph);
+                    if constexpr (SPLIT) tmem_st8(ta + 32 + gp * 8, pl);
+                    tmem_st8(ta + 64 + gp * 8, dh);
+                    if constexpr (SPLIT) tmem_st8(ta + 96 + gp * 8, dlo);
                 }
-                fence_proxy_async_smem();
+                tmem_st_wait();
+                tc_fence_before();
                 mbar_arrive(&bb.ds_full);
                 ++i;
             }
@@ -438,16 +464,17 @@ struct CfgQ {
     static constexpr uint32_t kTile = TM * D * 2;   // Q or dO tile
     static constexpr uint32_t kBlk = TB * D * 2;    // K_J or V_J block
     static constexpr uint32_t kStage = 2 * kBlk;
-    static constexpr uint32_t kPT = TM * TB * 2;    // dS tile (bf16)
     static constexpr uint32_t offQ = 0;
     static constexpr uint32_t offO = offQ + kTile;
     static constexpr uint32_t offSt = offO + kTile;  // 2 stages of K_J, V_J
-    static constexpr uint32_t offP = offSt + 2 * kStage;  // dS hi, dS lo
-    static constexpr uint32_t offBar = offP + 2 * kPT;
+    static constexpr uint32_t offBar = offSt + 2 * kStage;
+    // TMEM: S and dP double buffers, dQ, and the A tiles of the dQ MMA (dS hi, dS lo: 2 x 32 columns)
     static constexpr uint32_t colS = 0;
     static constexpr uint32_t colDP = 128;
     static constexpr uint32_t colDQ = 256;
+    static constexpr uint32_t colA = 256 + D;
     static constexpr uint32_t tmemCols = 512;
+    static_assert(colA + 64 <= tmemCols, "TMEM budget");
 };
 
 template <int D, int MODE, bool SPLIT>
@@ -509,7 +536,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sQ = smem_u32(smem + C::offQ);
     const uint32_t sO = smem_u32(smem + C::offO);
     const uint32_t sSt = smem_u32(smem + C::offSt);
-    const uint32_t sP = smem_u32(smem + C::offP);
 
     if (warp == 5) {
         if (lane == 0) {
@@ -575,11 +601,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < TB / 16; ++kk) {
                     const uint64_t dkb = sdesc_sw128(kb + kk * 2048, TB * 128, 1024);
-                    const uint64_t dsh = sdesc_sw128(sP + 0 * C::kPT + kk * 32, 16, 1024);
-                    const uint64_t dsl = sdesc_sw128(sP + 1 * C::kPT + kk * 32, 16, 1024);
+                    const uint32_t ta = tmem + C::colA + kk * 8;
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-                    mma_bf16_ss(tmem + C::colDQ, dsh, dkb, idG, acc);
-                    if constexpr (SPLIT) mma_bf16_ss(tmem + C::colDQ, dsl, dkb, idG, 1u);
+                    mma_bf16_ts(tmem + C::colDQ, ta, dkb, idG, acc);
+                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDQ, ta + 32, dkb, idG, 1u);
                 }
                 mma_commit(&bb.ds_empty);
                 mma_commit(&bb.q_empty[st]);
@@ -626,26 +651,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bb.s_empty[sb]);
                 const int j0 = J * TB;
                 const bool full = qvalid && (j0 + TB <= a.n) && (!a.causal || j0 + TB - 1 <= q0);
-                float dsv[TB];
-#pragma unroll
-                for (int c = 0; c < TB; ++c) {
-                    const int kj = j0 + c;
-                    const bool okc = full || (qvalid && kj < a.n && (!a.causal || kj <= row));
-                    float p, u;
-                    pointwise<MODE>(sv[c], stat, a.cz, a.k, okc, p, u);
-                    dsv[c] = u * (dpv[c] - dl);
-                }
                 ok = __all_sync(0xffffffffu, wait_bounded(&bb.ds_empty, (i & 1) ^ 1, abort_flag, a.status));
                 if (!ok) break;
+                const uint32_t ta = lane_base + C::colA;
 #pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    uint32_t dh[4], dlo[4];
-                    pack8<SPLIT>(dsv + 8 * g, dh, dlo);
-                    const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)g);
-                    st_shared_v4(sP + 0 * C::kPT + off, dh[0], dh[1], dh[2], dh[3]);
-                    if constexpr (SPLIT) st_shared_v4(sP + 1 * C::kPT + off, dlo[0], dlo[1], dlo[2], dlo[3]);
+                for (int gp = 0; gp < 4; ++gp) {
+                    uint32_t dh[8], dlo[8];
+                    bool anyx = (MODE == kModeSoftmax);
+                    if constexpr (MODE != kModeSoftmax) {
+                        float sm = sv[16 * gp];
+#pragma unroll
+                        for (int e = 1; e < 16; ++e) sm = fmaxf(sm, sv[16 * gp + e]);
+                        anyx = fmaf(sm, a.cz, -stat) > 0.f;
+                    }
+                    if (anyx) {
+#pragma unroll
+                    for (int q2 = 0; q2 < 8; ++q2) {
+                        float dd[2];
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int c = 16 * gp + 2 * q2 + e;
+                            const int kj = j0 + c;
+                            const bool okc = full || (qvalid && kj < a.n && (!a.causal || kj <= row));
+                            float p, u;
+                            pointwise<MODE>(sv[c], stat, a.cz, a.k, okc, p, u);
+                            dd[e] = u * (dpv[c] - dl);
+                        }
+                        split2<SPLIT>(dd, dh[q2], dlo[q2]);
+                    }
+                    } else {
+#pragma unroll
+                        for (int q2 = 0; q2 < 8; ++q2) dh[q2] = dlo[q2] = 0u;
+                    }
+                    tmem_st8(ta + gp * 8, dh);
+                    if constexpr (SPLIT) tmem_st8(ta + 32 + gp * 8, dlo);
                 }
-                fence_proxy_async_smem();
+                tmem_st_wait();
+                tc_fence_before();
                 mbar_arrive(&bb.ds_full);
                 ++i;
             }

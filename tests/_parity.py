@@ -52,6 +52,16 @@ def check_mask(mask_gpu_words, bits_ref, bmax_ref, where=""):
     return int((g != bits_ref).sum())
 
 
+def grad_xmin(tau):
+    """Support entries closer than this to tau* make an alpha > 2 gradient row unresolvable in float32.
+
+    With float32 scores off by dz ~ 3e-7 |tau|, dS = u (g - delta), u = x^(k-1) = x^(-1/2) (alpha = 3),
+    moves by ~0.5 dz x^(-3/2) |g - delta|; scaled by |q| / sqrt(d) (~12 / 8 here) this stays below the
+    2e-2 bound for x > (1e-4 |tau|)^(2/3). A factor 2 of margin on x is taken.
+    """
+    return 2.0 * (1e-4 * np.maximum(1.0, np.abs(tau))) ** (2.0 / 3.0)
+
+
 def conditioning(arr, alpha, causal, xmin=1e-2, flip=0.0):
     """Rows with an entry close to the support boundary, and the key columns those rows touch.
 
@@ -78,7 +88,8 @@ def conditioning(arr, alpha, causal, xmin=1e-2, flip=0.0):
                 tau = oe.tau_bisect(z, valid, alpha)
                 x = np.where(valid, z - tau[:, None], -1.0)
                 sup = x > 0
-                near = sup & (x < xmin)
+                xm = grad_xmin(tau)[:, None] if xmin == "grad" else xmin
+                near = sup & (x < xm)
                 if flip > 0:
                     near |= valid & (np.abs(z - tau[:, None]) < flip * np.maximum(1.0, np.abs(tau))[:, None])
                 br = near.any(axis=1)

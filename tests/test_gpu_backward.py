@@ -53,7 +53,7 @@ def test_bwd_small(torch_cuda, alpha, causal):
 # of tau (flip), alpha > 2 rows with a support entry below 1e-2 are reported and left out of the gradient
 # comparison; alpha > 2 rows with a support entry below 1e-4 are left out of the O comparison.
 GRAD_FLIP = 2e-6
-GRAD_XMIN = 1e-2
+GRAD_XMIN = "grad"  # per-row bound from _parity.grad_xmin
 FWD_XMIN = 1e-4
 
 
