@@ -177,7 +177,7 @@ __device__ __forceinline__ void hist_add(const HistRow& h, float a, float cbin, 
 // threshold are dropped; if that leaves it more than half full, the row is marked overflowed (it falls
 // back to sweeps) so that the pruning work stays amortised O(1) per entry.
 // ---------------------------------------------------------------------------------------------
-constexpr int kStashCap = 64;
+constexpr int kStashCap = 128;
 
 struct Stash {
     int n;

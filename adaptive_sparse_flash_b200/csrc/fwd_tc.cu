@@ -31,9 +31,8 @@ constexpr int BM = 128;           // query rows per tile
 constexpr int BN = 64;            // keys per block (= mask block)
 constexpr int NVS = 2;            // V ring stages
 constexpr int kThreads = 192;
-constexpr uint32_t kRowBufStride = 68;  // floats per row of the rare-path buffer (16-byte aligned, no conflicts)
-// dense sweep: histogram (u16, 64 KB) + stash (32 KB) + rare-path row buffer (34 KB); the V ring after it
-constexpr uint32_t kHistBytes = 256u * BM * 2u + kStashCap * BM * 4u + BM * kRowBufStride * 4u;
+// dense sweep: histogram (u16, 64 KB) + stash (64 KB); the V ring after it
+constexpr uint32_t kHistBytes = 256u * BM * 2u + kStashCap * BM * 4u;
 
 template <int D>
 struct Cfg {
@@ -95,9 +94,10 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
     return r;
 }
 
-// Out-of-line path of the dense sweep, taken when a row's stash is nearly full: drop the entries that
-// fell below the threshold; if the stash stays more than half full, the row switches to streaming its
-// histogram (its stash is binned now) and is marked overflowed. Returns the new stash count, or -1.
+// Out-of-line path of the dense sweep, taken when a row's stash may not hold another block: drop the
+// entries that fell below the threshold; if the stash stays more than half full, the row switches to
+// streaming its histogram (its stash is binned now) and is marked overflowed. Returns the new stash
+// count, or -1.
 static __device__ __noinline__ int stash_room(int n, HistRow& h, float* stash, uint16_t* hist, int r, float m_run,
                                               float thr, float cbin, int bins, int init_mode) {
     int j = 0;
@@ -116,7 +116,7 @@ static __device__ __noinline__ int stash_room(int n, HistRow& h, float* stash, u
 }
 
 // Streaming path for a row whose stash overflowed: bin this block's entries above the threshold
-// (rolled loop over the row's scores, staged in shared memory).
+// (rolled loop over the row's scores, staged in the row's now unused stash slots, rb[e * 128]).
 static __device__ __noinline__ void stream_block(HistRow& h, const float* rb, uint32_t gflag, float thr, float cbin,
                                                  int bins, int init_mode, uint16_t* hist, int r) {
     if (init_mode != 0) return;
@@ -124,7 +124,7 @@ static __device__ __noinline__ void stream_block(HistRow& h, const float* rb, ui
         const int g = __ffs(gflag) - 1;
         gflag &= gflag - 1;
         for (int e = 0; e < 8; ++e) {
-            const float v = rb[8 * g + e];
+            const float v = rb[(8 * g + e) * kTileRows];
             if (v > thr) hist_add(h, v, cbin, bins, hist, r);
         }
     }
@@ -151,7 +151,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* mrow = next + W;                                   // [2][W]
     uint16_t* hist = reinterpret_cast<uint16_t*>(smem + C::offU);                 // [256][128] u16
     float* stash = reinterpret_cast<float*>(smem + C::offU + 256 * BM * 2);        // [kStashCap][128]
-    float* rowbuf = stash + kStashCap * BM;                                        // [128][kRowBufStride]
     uint32_t* live_all = mrow + 2 * W;                                             // [128][kLiveStride]
 
     const SolveParams sp = a.sp;
@@ -423,48 +422,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (ovf && sp.init_mode == 0) hist_raise(h, amax, sp.cbin, sp.inv_cz, sp.bins);
             }
             const bool any = amax > thr;
-            if (any) {
-                if (!ovf) {
+            if (__any_sync(0xffffffffu, any)) {
+                // make room for a whole block first (at most once per block, out of line)
+                const bool room = any && !ovf && nst > kStashCap - BN;
+                if (__any_sync(0xffffffffu, room)) {
+                    if (room) {
+                        nst = stash_room(nst, h, stash, hist, r, m_run, thr, sp.cbin, sp.bins, sp.init_mode);
+                        if (nst < 0) { ovf = true; nst = 0; }
+                    }
+                }
+                // stash path, warp-uniform per group; predicated stores inside
 #pragma unroll
-                    for (int g = 0; g < 8; ++g) {
-                        if (gm[g] > thr) {
-                            if (nst > kStashCap - 8) {
-                                nst = stash_room(nst, h, stash, hist, r, m_run, thr, sp.cbin, sp.bins, sp.init_mode);
-                                if (nst < 0) { ovf = true; nst = 0; }
-                            }
-                            if (!ovf) {
+                for (int g = 0; g < 8; ++g) {
+                    const bool fl = !ovf && gm[g] > thr;
+                    if (__any_sync(0xffffffffu, fl)) {
 #pragma unroll
-                                for (int e = 0; e < 8; ++e) {
-                                    const float v = vbuf[8 * g + e];
-                                    if (v > thr) {
-                                        stash[nst * BM + r] = v;
-                                        ++nst;
-                                    }
-                                }
-                            } else {
-                                // switched to streaming in this block: bin the rest of it
-                                uint32_t gflag = 0u;
-#pragma unroll
-                                for (int g2 = 0; g2 < 8; ++g2) gflag |= (g2 >= g && gm[g2] > thr ? 1u : 0u) << g2;
-                                float* rb = rowbuf + r * kRowBufStride;
-#pragma unroll
-                                for (int c = 0; c < BN; c += 4)
-                                    *reinterpret_cast<float4*>(rb + c) =
-                                        make_float4(vbuf[c], vbuf[c + 1], vbuf[c + 2], vbuf[c + 3]);
-                                stream_block(h, rb, gflag, thr, sp.cbin, sp.bins, sp.init_mode, hist, r);
-                                break;
-                            }
+                        for (int e = 0; e < 8; ++e) {
+                            const float v = vbuf[8 * g + e];
+                            const bool q = fl && v > thr;
+                            if (q) stash[nst * BM + r] = v;
+                            nst += q ? 1 : 0;
                         }
                     }
-                } else {
-                    uint32_t gflag = 0u;
+                }
+                // rows that stream their histogram: rolled loop over the block's flagged groups
+                const bool strm = any && ovf && sp.init_mode == 0;
+                if (__any_sync(0xffffffffu, strm)) {
+                    if (strm) {
+                        uint32_t gflag = 0u;
 #pragma unroll
-                    for (int g = 0; g < 8; ++g) gflag |= (gm[g] > thr ? 1u : 0u) << g;
-                    float* rb = rowbuf + r * kRowBufStride;
+                        for (int g = 0; g < 8; ++g) gflag |= (gm[g] > thr ? 1u : 0u) << g;
 #pragma unroll
-                    for (int c = 0; c < BN; c += 4)
-                        *reinterpret_cast<float4*>(rb + c) = make_float4(vbuf[c], vbuf[c + 1], vbuf[c + 2], vbuf[c + 3]);
-                    stream_block(h, rb, gflag, thr, sp.cbin, sp.bins, sp.init_mode, hist, r);
+                        for (int c = 0; c < BN; ++c) stash[c * BM + r] = vbuf[c];
+                        stream_block(h, stash + r, gflag, thr, sp.cbin, sp.bins, sp.init_mode, hist, r);
+                    }
                 }
             }
             const uint32_t ball = __ballot_sync(0xffffffffu, any);
