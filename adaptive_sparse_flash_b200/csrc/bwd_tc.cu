@@ -28,10 +28,16 @@
 namespace eattn {
 namespace {
 
+// K-major operands (128-byte rows, 8-row groups 1024 bytes apart) and MN-major operands stored as
+// 64-column boxes of 64 rows (next 64 columns 8 KB further; next 8 rows 1024 bytes further)
+constexpr uint64_t kDescK = sdesc_sw128_fields(16, 1024);
+constexpr uint64_t kDescMN = sdesc_sw128_fields(64 * 128, 1024);
+
 constexpr int kThreads = 192;
 constexpr int TM = 128;  // rows of the tile owned by a CTA
 constexpr int TB = 64;   // rows of the blocks it walks
 constexpr int kModeSoftmax = 3;
+constexpr int NST = 4;   // stages of the operand ring that a CTA walks (Q_I/dO_I or K_J/V_J)
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
     asm volatile(
@@ -144,10 +150,11 @@ struct CfgKV {
     static constexpr uint32_t kStage = 2 * kBlk + 1024;  // Q_I, dO_I, stat[64], delta[64] (+ pad)
     static constexpr uint32_t offK = 0;
     static constexpr uint32_t offV = offK + kTile;
-    static constexpr uint32_t offSt = offV + kTile;               // 2 stages
-    static constexpr uint32_t offBar = offSt + 2 * kStage;
-    // TMEM: S^T and dP^T (double-buffered at d = 64), dV, dK, and the A tiles of the gradient MMAs
-    // (P^T hi, P^T lo, dS^T hi, dS^T lo: 4 x 32 columns, bf16 pairs), read by tcgen05.mma from TMEM.
+    static constexpr uint32_t offSt = offV + kTile;               // NST stages
+    static constexpr uint32_t offBar = offSt + NST * kStage;
+    // TMEM: S^T and dP^T (double-buffered at d = 64), dV, dK, and the A operands of the gradient MMAs,
+    // read by tcgen05.mma from TMEM: per K step of 16 query rows 32 columns [P^T hi | P^T lo | dS^T hi |
+    // dS^T lo], 8 columns (16 bf16) each.
     static constexpr int NSB = (D == 64) ? 2 : 1;
     static constexpr uint32_t colS = 0;
     static constexpr uint32_t colDP = NSB * TB;
@@ -160,7 +167,7 @@ struct CfgKV {
 
 struct BarsKV {
     uint64_t kv_full;
-    uint64_t q_full[2], q_empty[2];
+    uint64_t q_full[NST], q_empty[NST];
     uint64_t s_full[2], s_empty[2];
     uint64_t ds_full, ds_empty;
     uint64_t acc_full;
@@ -192,10 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         mbar_init(&bb.kv_full, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bb.q_full[i], 1); mbar_init(&bb.q_empty[i], 1);
-            mbar_init(&bb.s_full[i], 1); mbar_init(&bb.s_empty[i], TM);
-        }
+        for (int i = 0; i < NST; ++i) { mbar_init(&bb.q_full[i], 1); mbar_init(&bb.q_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&bb.s_full[i], 1); mbar_init(&bb.s_empty[i], TM); }
         mbar_init(&bb.ds_full, TM);
         mbar_init(&bb.ds_empty, 1);
         mbar_init(&bb.acc_full, 1);
@@ -246,8 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 while (bits && ok) {
                     const int I = w * 32 + __ffs(bits) - 1;
                     bits &= bits - 1;
-                    const uint32_t st = i & 1;
-                    if (!(ok = wait_bounded(&bb.q_empty[st], ((i >> 1) & 1) ^ 1, abort_flag, a.status, true))) break;
+                    const uint32_t st = i % NST;
+                    if (!(ok = wait_bounded(&bb.q_empty[st], ((i / NST) & 1) ^ 1, abort_flag, a.status, true))) break;
                     unsigned char* base = smem + C::offSt + st * C::kStage;
                     mbar_arrive_expect_tx(&bb.q_full[st], 2 * C::kBlk + 512);
                     for (int c = 0; c < D / 64; ++c) {
@@ -260,7 +265,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok) {
-                for (uint32_t j = (i > 2 ? i - 2 : 0); j < i; ++j) wait_drain(&bb.q_full[j & 1], (j >> 1) & 1, 100000000ull);
+                for (uint32_t j = (i > NST ? i - NST : 0); j < i; ++j) wait_drain(&bb.q_full[j % NST], (j / NST) & 1, 100000000ull);
                 wait_drain(&bb.kv_full, 0, 100000000ull);
             }
         }
@@ -272,18 +277,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             uint32_t i = 0;
             auto issue_S = [&](uint32_t idx) -> bool {
-                const uint32_t st = idx & 1, sb = idx % C::NSB;
-                if (!wait_bounded(&bb.q_full[st], (idx >> 1) & 1, abort_flag, a.status, true)) return false;
+                const uint32_t st = idx % NST, sb = idx % C::NSB;
+                if (!wait_bounded(&bb.q_full[st], (idx / NST) & 1, abort_flag, a.status, true)) return false;
                 if (!wait_bounded(&bb.s_empty[sb], ((idx / C::NSB) & 1) ^ 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t qb = sSt + st * C::kStage, ob = qb + C::kBlk;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t sub = kk >> 2, off = (kk & 3) * 32;
-                    const uint64_t dk = sdesc_sw128(sK + sub * (TM * 128) + off, 16, 1024);
-                    const uint64_t dq = sdesc_sw128(qb + sub * (TB * 128) + off, 16, 1024);
-                    const uint64_t dv = sdesc_sw128(sV + sub * (TM * 128) + off, 16, 1024);
-                    const uint64_t dd = sdesc_sw128(ob + sub * (TB * 128) + off, 16, 1024);
+                    const uint64_t dk = sdesc_at(kDescK, sK + sub * (TM * 128) + off);
+                    const uint64_t dq = sdesc_at(kDescK, qb + sub * (TB * 128) + off);
+                    const uint64_t dv = sdesc_at(kDescK, sV + sub * (TM * 128) + off);
+                    const uint64_t dd = sdesc_at(kDescK, ob + sub * (TB * 128) + off);
                     mma_bf16_ss(tmem + C::colS + sb * TB, dk, dq, idS, kk > 0);
                     mma_bf16_ss(tmem + C::colDP + sb * TB, dv, dd, idS, kk > 0);
                 }
@@ -291,20 +296,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             auto issue_G = [&](uint32_t idx, bool first) -> bool {
-                const uint32_t st = idx & 1;
+                const uint32_t st = idx % NST;
                 if (!wait_bounded(&bb.ds_full, idx & 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t qb = sSt + st * C::kStage, ob = qb + C::kBlk;
 #pragma unroll
                 for (int kk = 0; kk < TB / 16; ++kk) {
-                    const uint64_t dob = sdesc_sw128(ob + kk * 2048, TB * 128, 1024);
-                    const uint64_t dqb = sdesc_sw128(qb + kk * 2048, TB * 128, 1024);
-                    const uint32_t ta = tmem + C::colA + kk * 8;  // 16 query rows = 8 TMEM columns
+                    const uint64_t dob = sdesc_at(kDescMN, ob + kk * 2048);
+                    const uint64_t dqb = sdesc_at(kDescMN, qb + kk * 2048);
+                    const uint32_t ta = tmem + C::colA + 32 * kk;  // this K step's operands
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
                     mma_bf16_ts(tmem + C::colDV, ta + 0, dob, idG, acc);
-                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDV, ta + 32, dob, idG, 1u);
-                    mma_bf16_ts(tmem + C::colDK, ta + 64, dqb, idG, acc);
-                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDK, ta + 96, dqb, idG, 1u);
+                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDV, ta + 8, dob, idG, 1u);
+                    mma_bf16_ts(tmem + C::colDK, ta + 16, dqb, idG, acc);
+                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDK, ta + 24, dqb, idG, 1u);
                 }
                 mma_commit(&bb.ds_empty);
                 mma_commit(&bb.q_empty[st]);
@@ -335,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (bits) {
                 const int I = w * 32 + __ffs(bits) - 1;
                 bits &= bits - 1;
-                const uint32_t sb = i % C::NSB, st = i & 1;
+                const uint32_t sb = i % C::NSB, st = i % NST;
                 ok = __all_sync(0xffffffffu, wait_bounded(&bb.s_full[sb], (i / C::NSB) & 1, abort_flag, a.status));
                 if (!ok) break;
                 tc_fence_after();
@@ -348,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&bb.s_empty[sb]);
                 // the row statistics of block I arrived with its Q / dO stage
-                ok = __all_sync(0xffffffffu, wait_bounded(&bb.q_full[st], (i >> 1) & 1, abort_flag, a.status));
+                ok = __all_sync(0xffffffffu, wait_bounded(&bb.q_full[st], (i / NST) & 1, abort_flag, a.status));
                 if (!ok) break;
                 const float* stat = reinterpret_cast<const float*>(smem + C::offSt + st * C::kStage + 2 * C::kBlk);
                 const float* dl = stat + 64;
@@ -361,7 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // P^T and dS^T rows for this key against the 64 query rows of block I, 16 columns at a time
 #pragma unroll
                 for (int gp = 0; gp < 4; ++gp) {
-                    uint32_t ph[8], pl[8], dh[8], dlo[8];
+                    uint32_t ks[32];  // [P^T hi 8 | P^T lo 8 | dS^T hi 8 | dS^T lo 8]
+                    uint32_t* ph = ks;
+                    uint32_t* pl = ks + 8;
+                    uint32_t* dh = ks + 16;
+                    uint32_t* dlo = ks + 24;
                     float st16[16], dl16[16];
 #pragma unroll
                     for (int i4 = 0; i4 < 4; ++i4) {  // broadcast loads of the 16 columns' statistics
@@ -400,10 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int q2 = 0; q2 < 8; ++q2) ph[q2] = pl[q2] = dh[q2] = dlo[q2] = 0u;
                     }
-                    tmem_st8(ta + 0 + gp * 8, ph);
-                    if constexpr (SPLIT) tmem_st8(ta + 32 + gp * 8, pl);
-                    tmem_st8(ta + 64 + gp * 8, dh);
-                    if constexpr (SPLIT) tmem_st8(ta + 96 + gp * 8, dlo);
+                    tmem_st32(ta + 32 * gp, ks);
                 }
                 tmem_st_wait();
                 tc_fence_before();
@@ -466,9 +472,10 @@ struct CfgQ {
     static constexpr uint32_t kStage = 2 * kBlk;
     static constexpr uint32_t offQ = 0;
     static constexpr uint32_t offO = offQ + kTile;
-    static constexpr uint32_t offSt = offO + kTile;  // 2 stages of K_J, V_J
-    static constexpr uint32_t offBar = offSt + 2 * kStage;
-    // TMEM: S and dP double buffers, dQ, and the A tiles of the dQ MMA (dS hi, dS lo: 2 x 32 columns)
+    static constexpr uint32_t offSt = offO + kTile;  // NST stages of K_J, V_J
+    static constexpr uint32_t offBar = offSt + NST * kStage;
+    // TMEM: S and dP double buffers, dQ, and the A operands of the dQ MMA: per K step of 16 keys 16
+    // columns [dS hi | dS lo], 8 columns each
     static constexpr uint32_t colS = 0;
     static constexpr uint32_t colDP = 128;
     static constexpr uint32_t colDQ = 256;
@@ -499,10 +506,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         mbar_init(&bb.kv_full, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bb.q_full[i], 1); mbar_init(&bb.q_empty[i], 1);
-            mbar_init(&bb.s_full[i], 1); mbar_init(&bb.s_empty[i], TM);
-        }
+        for (int i = 0; i < NST; ++i) { mbar_init(&bb.q_full[i], 1); mbar_init(&bb.q_empty[i], 1); }
+        for (int i = 0; i < 2; ++i) { mbar_init(&bb.s_full[i], 1); mbar_init(&bb.s_empty[i], TM); }
         mbar_init(&bb.ds_full, TM);
         mbar_init(&bb.ds_empty, 1);
         mbar_init(&bb.acc_full, 1);
@@ -552,8 +557,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 while (bits && ok) {
                     const int J = w * 32 + __ffs(bits) - 1;
                     bits &= bits - 1;
-                    const uint32_t st = i & 1;
-                    if (!(ok = wait_bounded(&bb.q_empty[st], ((i >> 1) & 1) ^ 1, abort_flag, a.status, true))) break;
+                    const uint32_t st = i % NST;
+                    if (!(ok = wait_bounded(&bb.q_empty[st], ((i / NST) & 1) ^ 1, abort_flag, a.status, true))) break;
                     unsigned char* base = smem + C::offSt + st * C::kStage;
                     mbar_arrive_expect_tx(&bb.q_full[st], 2 * C::kBlk);
                     for (int c = 0; c < D / 64; ++c) {
@@ -564,7 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (!ok) {
-                for (uint32_t j = (i > 2 ? i - 2 : 0); j < i; ++j) wait_drain(&bb.q_full[j & 1], (j >> 1) & 1, 100000000ull);
+                for (uint32_t j = (i > NST ? i - NST : 0); j < i; ++j) wait_drain(&bb.q_full[j % NST], (j / NST) & 1, 100000000ull);
                 wait_drain(&bb.kv_full, 0, 100000000ull);
             }
         }
@@ -575,18 +580,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = wait_bounded(&bb.kv_full, 0, abort_flag, a.status, true);
             tc_fence_after();
             auto issue_S = [&](uint32_t idx) -> bool {
-                const uint32_t st = idx & 1, sb = idx & 1;
-                if (!wait_bounded(&bb.q_full[st], (idx >> 1) & 1, abort_flag, a.status, true)) return false;
+                const uint32_t st = idx % NST, sb = idx & 1;
+                if (!wait_bounded(&bb.q_full[st], (idx / NST) & 1, abort_flag, a.status, true)) return false;
                 if (!wait_bounded(&bb.s_empty[sb], ((idx >> 1) & 1) ^ 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t kb = sSt + st * C::kStage, vb = kb + C::kBlk;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t sub = kk >> 2, off = (kk & 3) * 32;
-                    const uint64_t dq = sdesc_sw128(sQ + sub * (TM * 128) + off, 16, 1024);
-                    const uint64_t dk = sdesc_sw128(kb + sub * (TB * 128) + off, 16, 1024);
-                    const uint64_t dd = sdesc_sw128(sO + sub * (TM * 128) + off, 16, 1024);
-                    const uint64_t dv = sdesc_sw128(vb + sub * (TB * 128) + off, 16, 1024);
+                    const uint64_t dq = sdesc_at(kDescK, sQ + sub * (TM * 128) + off);
+                    const uint64_t dk = sdesc_at(kDescK, kb + sub * (TB * 128) + off);
+                    const uint64_t dd = sdesc_at(kDescK, sO + sub * (TM * 128) + off);
+                    const uint64_t dv = sdesc_at(kDescK, vb + sub * (TB * 128) + off);
                     mma_bf16_ss(tmem + C::colS + sb * TB, dq, dk, idS, kk > 0);
                     mma_bf16_ss(tmem + C::colDP + sb * TB, dd, dv, idS, kk > 0);
                 }
@@ -594,17 +599,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 return true;
             };
             auto issue_G = [&](uint32_t idx, bool first) -> bool {
-                const uint32_t st = idx & 1;
+                const uint32_t st = idx % NST;
                 if (!wait_bounded(&bb.ds_full, idx & 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t kb = sSt + st * C::kStage;
 #pragma unroll
                 for (int kk = 0; kk < TB / 16; ++kk) {
-                    const uint64_t dkb = sdesc_sw128(kb + kk * 2048, TB * 128, 1024);
-                    const uint32_t ta = tmem + C::colA + kk * 8;
+                    const uint64_t dkb = sdesc_at(kDescMN, kb + kk * 2048);
+                    const uint32_t ta = tmem + C::colA + 16 * kk;
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
                     mma_bf16_ts(tmem + C::colDQ, ta, dkb, idG, acc);
-                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDQ, ta + 32, dkb, idG, 1u);
+                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDQ, ta + 8, dkb, idG, 1u);
                 }
                 mma_commit(&bb.ds_empty);
                 mma_commit(&bb.q_empty[st]);
@@ -656,7 +661,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t ta = lane_base + C::colA;
 #pragma unroll
                 for (int gp = 0; gp < 4; ++gp) {
-                    uint32_t dh[8], dlo[8];
+                    uint32_t ks[16];  // [dS hi 8 | dS lo 8]
+                    uint32_t* dh = ks;
+                    uint32_t* dlo = ks + 8;
                     bool anyx = (MODE == kModeSoftmax);
                     if constexpr (MODE != kModeSoftmax) {
                         float sm = sv[16 * gp];
@@ -683,8 +690,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int q2 = 0; q2 < 8; ++q2) dh[q2] = dlo[q2] = 0u;
                     }
-                    tmem_st8(ta + gp * 8, dh);
-                    if constexpr (SPLIT) tmem_st8(ta + 32 + gp * 8, dlo);
+                    tmem_st16(ta + 16 * gp, ks);
                 }
                 tmem_st_wait();
                 tc_fence_before();

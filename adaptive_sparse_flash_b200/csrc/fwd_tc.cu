@@ -27,9 +27,13 @@
 namespace eattn {
 namespace {
 
+// K-major operands (128-byte rows, 8-row groups 1024 bytes apart) and MN-major operands stored as
+// 64-column boxes of 64 rows (next 64 columns 8 KB further; next 8 rows 1024 bytes further)
+constexpr uint64_t kDescK = sdesc_sw128_fields(16, 1024);
+constexpr uint64_t kDescMN = sdesc_sw128_fields(64 * 128, 1024);
+
 constexpr int BM = 128;           // query rows per tile
 constexpr int BN = 64;            // keys per block (= mask block)
-constexpr int NVS = 2;            // V ring stages
 constexpr int kThreads = 192;
 // dense sweep: histogram (u16, 64 KB) + stash (64 KB); the V ring after it
 constexpr uint32_t kHistBytes = 256u * BM * 2u + kStashCap * BM * 4u;
@@ -37,6 +41,7 @@ constexpr uint32_t kHistBytes = 256u * BM * 2u + kStashCap * BM * 4u;
 template <int D>
 struct Cfg {
     static constexpr int NKS = (D == 64) ? 4 : 3;          // K ring stages
+    static constexpr int NVS = (D == 64) ? 6 : 4;          // V ring stages (inside the union region)
     static constexpr uint32_t kQBytes = BM * D * 2;        // 16 / 32 KB
     static constexpr uint32_t kKBytes = BN * D * 2;        // 8 / 16 KB per stage
     static constexpr uint32_t kPBytes = BM * BN * 2;       // 16 KB
@@ -46,12 +51,14 @@ struct Cfg {
     static constexpr uint32_t offU = offK + NKS * kKBytes;  // union region: histogram + stash, then V ring
     static constexpr uint32_t offV = offU;
     static_assert(NVS * kKBytes <= kHistBytes, "V ring must fit the union region");
+    static_assert(NVS <= 8, "barrier arrays");
     static constexpr uint32_t offSmall = offU + kHistBytes;
     static constexpr uint32_t tmemCols = 512;
     static constexpr uint32_t colO = 128;
     static constexpr uint32_t colOb = 128 + D;
     // P / U operands of the P V and U V MMAs live in TMEM (A operand from tensor memory): per buffer set
-    // 4 tiles of 128 lanes x 32 columns (64 bf16 per row): P high, P low, U high, U low.
+    // 128 columns, one group of 32 per K step of 16 keys: [P high | P low | U high | U low], 8 columns
+    // (16 bf16) each, so one 32-column store writes a K step of all four operands.
     static constexpr uint32_t colP = 128 + 2 * D;
     static_assert(colP + NPB * 128 <= tmemCols, "TMEM budget");
 };
@@ -59,7 +66,7 @@ struct Cfg {
 struct Small {
     uint64_t q_full;
     uint64_t k_full[4], k_empty[4];
-    uint64_t v_full[NVS], v_empty[NVS];
+    uint64_t v_full[8], v_empty[8];
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full[2], p_empty[2];
     uint64_t o_full;
@@ -167,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
         mbar_init(&sm.q_full, 1);
         for (int i = 0; i < C::NKS; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
-        for (int i = 0; i < NVS; ++i) { mbar_init(&sm.v_full[i], 1); mbar_init(&sm.v_empty[i], 1); }
+        for (int i = 0; i < C::NVS; ++i) { mbar_init(&sm.v_full[i], 1); mbar_init(&sm.v_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.s_full[i], 1); mbar_init(&sm.s_empty[i], BM);
             mbar_init(&sm.p_full[i], BM); mbar_init(&sm.p_empty[i], 1);
@@ -220,8 +227,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         64 * c, J * BN, bh);
                         ++lc;
                         if (kind == kSweepPV) {
-                            const uint32_t vs = vc % NVS;
-                            if (!(ok = wait_bounded(&sm.v_empty[vs], ((vc / NVS) & 1) ^ 1, abort_flag, a.status, true))) break;
+                            const uint32_t vs = vc % C::NVS;
+                            if (!(ok = wait_bounded(&sm.v_empty[vs], ((vc / C::NVS) & 1) ^ 1, abort_flag, a.status, true))) break;
                             mbar_arrive_expect_tx(&sm.v_full[vs], C::kKBytes);
                             for (int c = 0; c < D / 64; ++c)
                                 tma_load_3d(smem + C::offV + vs * C::kKBytes + c * (BN * 128), &tmV,
@@ -235,8 +242,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // drain copies still in flight before the CTA's shared memory is released
                 for (uint32_t i = (lc > (uint32_t)C::NKS ? lc - C::NKS : 0); i < lc; ++i)
                     wait_drain(&sm.k_full[i % C::NKS], (i / C::NKS) & 1, 100000000ull);
-                for (uint32_t i = (vc > (uint32_t)NVS ? vc - NVS : 0); i < vc; ++i)
-                    wait_drain(&sm.v_full[i % NVS], (i / NVS) & 1, 100000000ull);
+                for (uint32_t i = (vc > (uint32_t)C::NVS ? vc - C::NVS : 0); i < vc; ++i)
+                    wait_drain(&sm.v_full[i % C::NVS], (i / C::NVS) & 1, 100000000ull);
                 wait_drain(&sm.q_full, 0, 100000000ull);
             }
         }
@@ -257,8 +264,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t sub = kk >> 2, off = (kk & 3) * 32;
-                    const uint64_t da = sdesc_sw128(sQ + sub * (BM * 128) + off, 16, 1024);
-                    const uint64_t db = sdesc_sw128(kbase + sub * (BN * 128) + off, 16, 1024);
+                    const uint64_t da = sdesc_at(kDescK, sQ + sub * (BM * 128) + off);
+                    const uint64_t db = sdesc_at(kDescK, kbase + sub * (BN * 128) + off);
                     mma_bf16_ss(tmem + sb * BN, da, db, idS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&sm.s_full[sb]);
@@ -269,22 +276,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             };
             auto issue_PV = [&](bool first) -> bool {
                 const uint32_t pb = pc % C::NPB;
-                const uint32_t vs = vc % NVS;
+                const uint32_t vs = vc % C::NVS;
                 if (!wait_bounded(&sm.p_full[pb], (pc / C::NPB) & 1, abort_flag, a.status, true)) return false;
-                if (!wait_bounded(&sm.v_full[vs], (vc / NVS) & 1, abort_flag, a.status, true)) return false;
+                if (!wait_bounded(&sm.v_full[vs], (vc / C::NVS) & 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
                 const uint32_t vbase = sV0 + vs * C::kKBytes;
                 const uint32_t tp = tmem + C::colP + pb * 128;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk) {
-                    const uint64_t dv = sdesc_sw128(vbase + kk * 2048, BN * 128, 1024);
+                    const uint64_t dv = sdesc_at(kDescMN, vbase + kk * 2048);
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
                     // P = P_hi + P_lo and U = U_hi + U_lo (two bf16 terms each) keep P V and U V accurate
                     // to ~16 mantissa bits; each K step of 16 keys is 8 TMEM columns of the A tile
-                    mma_bf16_ts(tmem + C::colO, tp + 0 + kk * 8, dv, idPV, acc);
-                    mma_bf16_ts(tmem + C::colO, tp + 32 + kk * 8, dv, idPV, 1u);
-                    mma_bf16_ts(tmem + C::colOb, tp + 64 + kk * 8, dv, idPV, acc);
-                    mma_bf16_ts(tmem + C::colOb, tp + 96 + kk * 8, dv, idPV, 1u);
+                    mma_bf16_ts(tmem + C::colO, tp + 32 * kk + 0, dv, idPV, acc);
+                    mma_bf16_ts(tmem + C::colO, tp + 32 * kk + 8, dv, idPV, 1u);
+                    mma_bf16_ts(tmem + C::colOb, tp + 32 * kk + 16, dv, idPV, acc);
+                    mma_bf16_ts(tmem + C::colOb, tp + 32 * kk + 24, dv, idPV, 1u);
                 }
                 mma_commit(&sm.p_empty[pb]);
                 mma_commit(&sm.v_empty[vs]);
@@ -568,8 +575,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t tp = lane_base + C::colP + pb * 128;
 #pragma unroll
                     for (int gp = 0; gp < 4; ++gp) {
-                        // two groups of 8 keys = 8 TMEM columns of each of the four A tiles
-                        uint32_t ph[8], pl[8], uh[8], ul[8];
+                        // two groups of 8 keys = one K step: 8 columns of each of the four operands
+                        uint32_t ks[32];  // [P high 8 | P low 8 | U high 8 | U low 8]
+                        uint32_t* ph = ks;
+                        uint32_t* pl = ks + 8;
+                        uint32_t* uh = ks + 16;
+                        uint32_t* ul = ks + 24;
 #pragma unroll
                         for (int q8 = 0; q8 < 2; ++q8) {
                             const int g = 2 * gp + q8;
@@ -616,10 +627,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 for (int w = q8 * 4; w < q8 * 4 + 4; ++w) ph[w] = pl[w] = uh[w] = ul[w] = 0u;
                             }
                         }
-                        tmem_st8(tp + 0 + gp * 8, ph);
-                        tmem_st8(tp + 32 + gp * 8, pl);
-                        tmem_st8(tp + 64 + gp * 8, uh);
-                        tmem_st8(tp + 96 + gp * 8, ul);
+                        tmem_st32(tp + 32 * gp, ks);
                     }
                     tmem_st_wait();
                     mbar_arrive(&sm.p_full[pb]);

@@ -17,6 +17,11 @@
 namespace eattn {
 namespace {
 
+// K-major operands (128-byte rows, 8-row groups 1024 bytes apart) and MN-major operands stored as
+// 64-column boxes of 64 rows (next 64 columns 8 KB further; next 8 rows 1024 bytes further)
+constexpr uint64_t kDescK = sdesc_sw128_fields(16, 1024);
+constexpr uint64_t kDescMN = sdesc_sw128_fields(64 * 128, 1024);
+
 constexpr int BM = 128, BN = 64, kThreads = 192, NST = 3;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -44,18 +49,6 @@ struct BarsS {
     uint32_t tmem_base;
     int abort_flag;
 };
-
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -138,8 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t sub = kk >> 2, off = (kk & 3) * 32;
-                    mma_bf16_ss(tmem + sb * BN, sdesc_sw128(sQ + sub * (BM * 128) + off, 16, 1024),
-                                sdesc_sw128(kb + sub * (BN * 128) + off, 16, 1024), idS, kk > 0);
+                    mma_bf16_ss(tmem + sb * BN, sdesc_at(kDescK, sQ + sub * (BM * 128) + off),
+                                sdesc_at(kDescK, kb + sub * (BN * 128) + off), idS, kk > 0);
                 }
                 mma_commit(&bb.s_full[sb]);
                 return true;
@@ -151,8 +144,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t vb = sSt + st * C::kStage + C::kBlk;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_bf16_ss(tmem + C::colO, sdesc_sw128(sP + pb * C::kPBytes + kk * 32, 16, 1024),
-                                sdesc_sw128(vb + kk * 2048, BN * 128, 1024), idPV, (J > 0 || kk > 0) ? 1u : 0u);
+                    mma_bf16_ss(tmem + C::colO, sdesc_at(kDescK, sP + pb * C::kPBytes + kk * 32),
+                                sdesc_at(kDescMN, vb + kk * 2048), idPV, (J > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&bb.p_empty[pb]);
                 mma_commit(&bb.kv_empty[st]);
                 mma_commit(&bb.pv_done[J & 1]);
