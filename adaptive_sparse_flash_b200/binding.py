@@ -36,6 +36,7 @@ EXPORTS = (
     "entmax_attn_selftest_timeout",
     "entmax_status_str",
     "entmax_attn_version",
+    "entmax_attn_fwd_noalloc",
 )
 
 
@@ -108,6 +109,9 @@ def lib() -> ctypes.CDLL:
     L.entmax_status_str.restype = ctypes.c_char_p
     L.entmax_attn_version.argtypes = []
     L.entmax_attn_version.restype = i
+    L.entmax_attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, op, vp]
+    L.entmax_attn_fwd_noalloc.restype = i
+
     _lib = L
     return L
 
@@ -206,6 +210,18 @@ def softmax_attn_bwd(Q, K, V, O, dO, lse, dQ, dK, dV, causal, opts: EntmaxOpts, 
                                 _ptr(dV), B, H, n, d, int(causal), _dtype_code(Q), ctypes.byref(opts),
                                 _stream(stream))
     _check(st, "softmax_attn_bwd")
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20  # size of the library's scratch array used by entmax_attn_fwd_noalloc
+
+
+def entmax_attn_fwd_noalloc(Q, K, V, O, tau, block_mask, alpha, causal, opts: EntmaxOpts | None = None, stream=None):
+    """Forward that allocates nothing: the library's fixed scratch array replaces the workspace."""
+    B, H, n, d = Q.shape
+    st = lib().entmax_attn_fwd_noalloc(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(tau), _ptr(block_mask),
+                                       B, H, n, d, float(alpha), int(causal), _dtype_code(Q),
+                                       None if opts is None else ctypes.byref(opts), _stream(stream))
+    _check(st, "entmax_attn_fwd_noalloc")
 
 
 def entmax_attn_check(stream=None) -> int:

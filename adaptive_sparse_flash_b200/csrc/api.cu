@@ -298,3 +298,63 @@ EATTN_API entmax_status softmax_attn_bwd(const void* Q, const void* K, const voi
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------------------
+// Forward without caller-provided workspace (no allocation at all).
+//
+// Some callers cannot allocate device memory: code that runs while a host framework owns the whole
+// device pool and exposes no allocator, or that must not call cudaMalloc on its path (it can
+// synchronise the device, and it is not allowed while a stream is being captured). For them the
+// forward can use a fixed scratch area that lives in the library image: a file-scope device array of
+// kStaticScratchBytes, which every GPU that loads the library keeps until the process exits. Host code
+// cannot use the array's name as a device address, so its address is looked up once per device.
+// ---------------------------------------------------------------------------------------------
+namespace eattn {
+namespace {
+
+constexpr size_t kStaticScratchBytes = (size_t)32 << 20;  // 32 MiB
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of the scratch array on the current device (looked up on the first call per device,
+// with that device current). Returns nullptr if the lookup fails.
+void* static_scratch_ptr() {
+    static void* cache[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr) return nullptr;
+        cache[dev] = p;
+    }
+    return cache[dev];
+}
+
+}  // namespace
+}  // namespace eattn
+
+extern "C" {
+
+EATTN_API entmax_status entmax_attn_fwd_noalloc(const void* Q, const void* K, const void* V, void* O, float* tau,
+                                                uint32_t* block_mask, int B, int H, int n, int d, float alpha,
+                                                int causal, entmax_dtype dt, const entmax_opts* opts, void* stream) {
+    entmax_opts o;
+    memset(&o, 0, sizeof(o));
+    if (opts) o = *opts;
+    const size_t need = entmax_attn_workspace_size(B, H, n, d, dt, &o);
+    if (need == 0) {
+        // let the regular checks name the problem (invalid or unsupported sizes)
+        o.workspace = nullptr;
+        o.workspace_bytes = 0;
+        Dims D;
+        const entmax_status st = check_dims(B, H, n, d, dt, &o, &D);
+        return st != ENTMAX_OK ? st : ENTMAX_ERR_INVALID;
+    }
+    if (need > kStaticScratchBytes) return ENTMAX_ERR_WORKSPACE;
+    void* scratch = static_scratch_ptr();
+    if (!scratch) return ENTMAX_ERR_CUDA;
+    o.workspace = scratch;
+    o.workspace_bytes = kStaticScratchBytes;
+    return entmax_attn_fwd(Q, K, V, O, tau, block_mask, B, H, n, d, alpha, causal, dt, &o, stream);
+}
+
+}  // extern "C"

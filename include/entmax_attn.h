@@ -114,6 +114,21 @@ entmax_status softmax_attn_bwd(const void* Q, const void* K, const void* V, cons
                                const float* lse, void* dQ, void* dK, void* dV, int B, int H, int n, int d,
                                int causal, entmax_dtype dt, const entmax_opts* opts, void* stream);
 
+/* Forward that allocates nothing and needs no workspace (the paper has no counterpart: this is for
+ * callers that cannot allocate device memory, e.g. code running inside a framework that owns the whole
+ * device pool, or paths that must not call cudaMalloc, which may synchronise and is not allowed during
+ * stream capture). Same arguments, outputs and checks as entmax_attn_fwd; opts may be NULL and any
+ * opts->workspace is ignored. The scratch lives in a 32 MiB (33554432-byte) device array inside the
+ * library, which every GPU that loads the library holds until exit; calls whose workspace
+ * (entmax_attn_workspace_size) would be larger return ENTMAX_ERR_WORKSPACE. The first call on
+ * each device looks up the array's device address (cudaGetSymbolAddress), so make that first call
+ * before any stream capture. All calls share the array and it keeps the last call's contents (no part
+ * of it needs to start at zero); calls that may overlap on the GPU (other streams, other host threads)
+ * race on it, and a later entmax_attn_bwd cannot use it: for training use entmax_attn_fwd. */
+entmax_status entmax_attn_fwd_noalloc(const void* Q, const void* K, const void* V, void* O, float* tau,
+                                      uint32_t* block_mask, int B, int H, int n, int d, float alpha, int causal,
+                                      entmax_dtype dt, const entmax_opts* opts, void* stream);
+
 /* Synchronises `stream`, then returns and clears the device status word of the current device:
  * ENTMAX_ERR_TIMEOUT if a kernel's bounded wait ran out since the last check, ENTMAX_ERR_CUDA if the
  * stream reports an error, else ENTMAX_OK. */
