@@ -56,6 +56,7 @@ class EntmaxStats(ctypes.Structure):
         ("candidate_blocks", ctypes.c_ulonglong),
         ("nonzero_blocks", ctypes.c_ulonglong),
         ("sweeps", ctypes.c_ulonglong),
+        ("overflow_rows", ctypes.c_ulonglong),
     ]
 
 
@@ -277,7 +278,7 @@ def backward(Q, K, V, fwd: EntmaxForward, dO, stream=None):
 def stats_dict(stats_tensor) -> dict:
     v = [int(x) for x in stats_tensor.cpu().tolist()]
     names = ["rows", "steps", "fallbacks"] + [f"step_hist_{i}" for i in range(9)] + \
-        ["causal_blocks", "candidate_blocks", "nonzero_blocks", "sweeps"]
+        ["causal_blocks", "candidate_blocks", "nonzero_blocks", "sweeps", "overflow_rows"]
     return dict(zip(names, v))
 
 

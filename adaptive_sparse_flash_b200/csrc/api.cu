@@ -91,6 +91,11 @@ struct Workspace {
     float* delta_pad;
     float* stat_pad;
     uint32_t* maskT;
+    uint32_t* maxbits;  // [8]: max |x| of Q, K, V (forward), dO (backward), as float bits
+    void* Qh;           // fp16 copies [BH][n][d] (f16.cu)
+    void* Kh;
+    void* Vh;
+    void* dOh;
     size_t bytes;
 };
 
@@ -110,6 +115,13 @@ Workspace layout(const Dims& D, void* base) {
     off = align256(off + rows_pad * sizeof(float));
     w.maskT = reinterpret_cast<uint32_t*>(p + off);
     off = align256(off + (size_t)D.B * D.H * D.nkb * D.nwq * sizeof(uint32_t));
+    w.maxbits = reinterpret_cast<uint32_t*>(p + off);
+    off = align256(off + 8 * sizeof(uint32_t));
+    void** h16[4] = {&w.Qh, &w.Kh, &w.Vh, &w.dOh};
+    for (int i = 0; i < 4; ++i) {
+        *h16[i] = p + off;
+        off = align256(off + rows * D.d * 2);
+    }
     w.bytes = off;
     return w;
 }
@@ -123,6 +135,21 @@ entmax_status check_workspace(const Dims& D, const entmax_opts* o, Workspace* w)
 }
 
 inline entmax_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ENTMAX_OK : ENTMAX_ERR_CUDA; }
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int v = 0;
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v < 1) v = 148;
+        cache[dev] = v;
+    }
+    return cache[dev];
+}
+
+// The fp16 forward (fwd_h.cu) serves bf16 inputs with d = 64 and alpha <= 2 (p and u in [0, 1]).
+inline bool use_f16_path(int d, float alpha) { return d == 64 && alpha <= 2.0f; }
 
 }  // namespace
 }  // namespace eattn
@@ -182,6 +209,18 @@ EATTN_API entmax_status entmax_attn_fwd(const void* Q, const void* K, const void
     cudaError_t e;
     if (dt == ENTMAX_FP32) {
         e = launch_fwd_simt(a, true, s);
+    } else if (use_f16_path(d, alpha)) {
+        F16Job job;
+        memset(&job, 0, sizeof(job));
+        job.src[0] = Q; job.src[1] = K; job.src[2] = V;
+        job.dst[0] = ws.Qh; job.dst[1] = ws.Kh; job.dst[2] = ws.Vh;
+        job.maxbits = ws.maxbits;
+        job.n16 = (size_t)B * H * n * d / 8;
+        job.count = 3;
+        a.Qh = ws.Qh; a.Kh = ws.Kh; a.Vh = ws.Vh; a.maxbits = ws.maxbits;
+        e = launch_to_f16(job, num_sms(), s);
+        if (e == cudaSuccess) e = launch_fwd_h(a, s);
+        if (e == cudaSuccess) e = launch_mask_transpose(block_mask, ws.maskT, B * H, D.nqb, D.nkb, D.nw, D.nwq, s);
     } else {
         e = launch_fwd_tc(a, s);
         if (e == cudaSuccess) e = launch_mask_transpose(block_mask, ws.maskT, B * H, D.nqb, D.nkb, D.nw, D.nwq, s);

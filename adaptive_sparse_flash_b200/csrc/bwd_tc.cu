@@ -289,8 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t dq = sdesc_at(kDescK, qb + sub * (TB * 128) + off);
                     const uint64_t dv = sdesc_at(kDescK, sV + sub * (TM * 128) + off);
                     const uint64_t dd = sdesc_at(kDescK, ob + sub * (TB * 128) + off);
-                    mma_bf16_ss(tmem + C::colS + sb * TB, dk, dq, idS, kk > 0);
-                    mma_bf16_ss(tmem + C::colDP + sb * TB, dv, dd, idS, kk > 0);
+                    mma_ss(tmem + C::colS + sb * TB, dk, dq, idS, kk > 0);
+                    mma_ss(tmem + C::colDP + sb * TB, dv, dd, idS, kk > 0);
                 }
                 mma_commit(&bb.s_full[sb]);
                 return true;
@@ -306,10 +306,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t dqb = sdesc_at(kDescMN, qb + kk * 2048);
                     const uint32_t ta = tmem + C::colA + 32 * kk;  // this K step's operands
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-                    mma_bf16_ts(tmem + C::colDV, ta + 0, dob, idG, acc);
-                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDV, ta + 8, dob, idG, 1u);
-                    mma_bf16_ts(tmem + C::colDK, ta + 16, dqb, idG, acc);
-                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDK, ta + 24, dqb, idG, 1u);
+                    mma_ts(tmem + C::colDV, ta + 0, dob, idG, acc);
+                    if constexpr (SPLIT) mma_ts(tmem + C::colDV, ta + 8, dob, idG, 1u);
+                    mma_ts(tmem + C::colDK, ta + 16, dqb, idG, acc);
+                    if constexpr (SPLIT) mma_ts(tmem + C::colDK, ta + 24, dqb, idG, 1u);
                 }
                 mma_commit(&bb.ds_empty);
                 mma_commit(&bb.q_empty[st]);
@@ -592,8 +592,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t dk = sdesc_at(kDescK, kb + sub * (TB * 128) + off);
                     const uint64_t dd = sdesc_at(kDescK, sO + sub * (TM * 128) + off);
                     const uint64_t dv = sdesc_at(kDescK, vb + sub * (TB * 128) + off);
-                    mma_bf16_ss(tmem + C::colS + sb * TB, dq, dk, idS, kk > 0);
-                    mma_bf16_ss(tmem + C::colDP + sb * TB, dd, dv, idS, kk > 0);
+                    mma_ss(tmem + C::colS + sb * TB, dq, dk, idS, kk > 0);
+                    mma_ss(tmem + C::colDP + sb * TB, dd, dv, idS, kk > 0);
                 }
                 mma_commit(&bb.s_full[sb]);
                 return true;
@@ -608,8 +608,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint64_t dkb = sdesc_at(kDescMN, kb + kk * 2048);
                     const uint32_t ta = tmem + C::colA + 16 * kk;
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-                    mma_bf16_ts(tmem + C::colDQ, ta, dkb, idG, acc);
-                    if constexpr (SPLIT) mma_bf16_ts(tmem + C::colDQ, ta + 8, dkb, idG, 1u);
+                    mma_ts(tmem + C::colDQ, ta, dkb, idG, acc);
+                    if constexpr (SPLIT) mma_ts(tmem + C::colDQ, ta + 8, dkb, idG, 1u);
                 }
                 mma_commit(&bb.ds_empty);
                 mma_commit(&bb.q_empty[st]);

@@ -7,6 +7,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -58,13 +59,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (for a thread that polls several barriers).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity. Returns false (and sets *abort) on timeout or
 // when another role of the CTA has already aborted.
 // `backoff`: the waiting thread sleeps between polls (exponentially, up to 256 ns), for the issuing warps
 // whose spinning would otherwise take issue slots from the compute warps on the same scheduler.
-static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
-                                                 bool backoff = false) {
-    if (mbar_try_wait(bar, parity)) return true;
+static __device__ __noinline__ bool wait_bounded_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                      int* status, bool backoff) {
     const uint64_t t0 = globaltimer();
     uint32_t ns = 8;
     for (uint32_t i = 0; i < kWaitIterCap; ++i) {
@@ -81,6 +94,14 @@ static __device__ __noinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
     *abort = 1;
     if (status) atomicExch(status, (int)ENTMAX_ERR_TIMEOUT);
     return false;
+}
+
+// Inline fast path (one poll); the polling loop stays out of line, so that the spills a call needs are
+// only paid when the wait actually blocks.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                             bool backoff = false) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bounded_slow(bar, parity, abort, status, backoff);
 }
 
 // Short bounded wait used while cleaning up after an abort: waits for copies still in flight.
@@ -137,8 +158,9 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulator (kind::f16).
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A[smem] * B[smem]^T, 16-bit inputs (bf16 or fp16, named by the instruction descriptor),
+// fp32 accumulator (kind::f16).
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -147,9 +169,9 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem]^T: A (M x 16 bf16 per instruction) read from tensor memory, one row
-// per lane, two bf16 per 32-bit column (element 2j in the low half).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A[tmem] * B[smem]^T: A (M x 16 16-bit elements per instruction) read from tensor memory,
+// one row per lane, two elements per 32-bit column (element 2j in the low half).
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
                                             uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -205,6 +227,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn, b
            | ((uint32_t)(M >> 4) << 24);   // M / 16
 }
 
+// Instruction descriptor, kind::f16 with fp16 A/B and fp32 D (A and B of one MMA share their type).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool a_mn, bool b_mn) {
+    return (1u << 4)                       // D format: f32; A and B format fields 0: f16
+           | ((a_mn ? 1u : 0u) << 15)
+           | ((b_mn ? 1u : 0u) << 16)
+           | ((uint32_t)(N >> 3) << 17)
+           | ((uint32_t)(M >> 4) << 24);
+}
+
 // Shared-memory matrix descriptor for a 128-byte-swizzled tile (the layout TMA writes with
 // CU_TENSOR_MAP_SWIZZLE_128B into a 1024-byte aligned buffer).
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
@@ -249,6 +280,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
         : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

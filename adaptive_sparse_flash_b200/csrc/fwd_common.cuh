@@ -27,9 +27,14 @@ struct FwdArgs {
     int causal;
     int ntiles;        // 128-row query tiles per head
     SolveParams sp;
+    // fp16 path (alpha <= 2, d = 64): fp16 copies of Q, K, V and their range exponents (f16.cu)
+    const void* Qh;
+    const void* Kh;
+    const void* Vh;
+    const uint32_t* maxbits;  // [3]: Q, K, V
 };
 
-enum SweepKind : int { kSweepDense = 0, kSweepRefine = 1, kSweepPV = 2, kSweepDone = 3 };
+enum SweepKind : int { kSweepDense = 0, kSweepRefine = 1, kSweepPV = 2, kSweepDone = 3, kSweepHist = 4 };
 
 // Number of allowed keys of query row `row`.
 __device__ __forceinline__ int allowed_keys(int row, int n, int causal) {
@@ -38,7 +43,7 @@ __device__ __forceinline__ int allowed_keys(int row, int n, int causal) {
 
 // Per-CTA statistics, reduced into entmax_stats at the end of a tile.
 struct TileStats {
-    uint32_t rows, steps, fallbacks, candidate_blocks, nonzero_blocks, causal_blocks, sweeps;
+    uint32_t rows, steps, fallbacks, candidate_blocks, nonzero_blocks, causal_blocks, sweeps, overflow_rows;
     uint32_t step_hist[kMaxSteps + 1];
 };
 
@@ -51,6 +56,7 @@ __device__ __forceinline__ void flush_stats(entmax_stats* g, const TileStats& t)
     atomicAdd(&g->nonzero_blocks, (unsigned long long)t.nonzero_blocks);
     atomicAdd(&g->causal_blocks, (unsigned long long)t.causal_blocks);
     atomicAdd(&g->sweeps, (unsigned long long)t.sweeps);
+    if (t.overflow_rows) atomicAdd(&g->overflow_rows, (unsigned long long)t.overflow_rows);
     for (int i = 0; i <= kMaxSteps; ++i)
         if (t.step_hist[i]) atomicAdd(&g->step_hist[i], (unsigned long long)t.step_hist[i]);
 }

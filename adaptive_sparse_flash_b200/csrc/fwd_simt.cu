@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
         a.tau[head + row] = s.tau;
         a.sum_u[head + row] = Su;
         if (a.steps) a.steps[head + row] = (uint8_t)s.steps;
+        if (sh.overflow) atomicAdd(&st.overflow_rows, 1u);
         atomicAdd(&st.rows, 1u);
         atomicAdd(&st.steps, (uint32_t)s.steps);
         atomicAdd(&st.fallbacks, (uint32_t)s.fallbacks);

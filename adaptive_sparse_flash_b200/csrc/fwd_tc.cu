@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sub = kk >> 2, off = (kk & 3) * 32;
                     const uint64_t da = sdesc_at(kDescK, sQ + sub * (BM * 128) + off);
                     const uint64_t db = sdesc_at(kDescK, kbase + sub * (BN * 128) + off);
-                    mma_bf16_ss(tmem + sb * BN, da, db, idS, kk > 0 ? 1u : 0u);
+                    mma_ss(tmem + sb * BN, da, db, idS, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&sm.s_full[sb]);
                 mma_commit(&sm.k_empty[ks]);
@@ -288,10 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
                     // P = P_hi + P_lo and U = U_hi + U_lo (two bf16 terms each) keep P V and U V accurate
                     // to ~16 mantissa bits; each K step of 16 keys is 8 TMEM columns of the A tile
-                    mma_bf16_ts(tmem + C::colO, tp + 32 * kk + 0, dv, idPV, acc);
-                    mma_bf16_ts(tmem + C::colO, tp + 32 * kk + 8, dv, idPV, 1u);
-                    mma_bf16_ts(tmem + C::colOb, tp + 32 * kk + 16, dv, idPV, acc);
-                    mma_bf16_ts(tmem + C::colOb, tp + 32 * kk + 24, dv, idPV, 1u);
+                    mma_ts(tmem + C::colO, tp + 32 * kk + 0, dv, idPV, acc);
+                    mma_ts(tmem + C::colO, tp + 32 * kk + 8, dv, idPV, 1u);
+                    mma_ts(tmem + C::colOb, tp + 32 * kk + 16, dv, idPV, acc);
+                    mma_ts(tmem + C::colOb, tp + 32 * kk + 24, dv, idPV, 1u);
                 }
                 mma_commit(&sm.p_empty[pb]);
                 mma_commit(&sm.v_empty[vs]);
@@ -719,6 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (nzb) atomicAdd(&sm.st.nonzero_blocks, nzb);
             if (cnd) atomicAdd(&sm.st.candidate_blocks, cnd);
             if (valid) {
+                if (sh.overflow) atomicAdd(&sm.st.overflow_rows, 1u);
                 atomicAdd(&sm.st.rows, 1u);
                 atomicAdd(&sm.st.steps, (uint32_t)s.steps);
                 atomicAdd(&sm.st.fallbacks, (uint32_t)s.fallbacks);
@@ -765,18 +766,27 @@ EncodeTiled get_encode() {
 
 }  // namespace
 
-// [BH, n, d] bf16 tensor, boxes of `rows` x 64 columns, 128B swizzle; zero fill past n.
-cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d, int rows) {
+// [BH, n, d] tensor of 16-bit elements, boxes of `rows` x 64 columns, 128B swizzle; zero fill past n.
+static cudaError_t make_tmap_16(CUtensorMap* map, const void* base, int BH, int n, int d, int rows,
+                                CUtensorMapDataType type) {
     EncodeTiled enc = get_encode();
     if (!enc) return cudaErrorNotSupported;
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)n, (cuuint64_t)BH};
     cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)n * d * 2};
     cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+    CUresult r = enc(map, type, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d, int rows) {
+    return make_tmap_16(map, base, BH, n, d, rows, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+}
+
+cudaError_t make_tmap_f16(CUtensorMap* map, const void* base, int BH, int n, int d, int rows) {
+    return make_tmap_16(map, base, BH, n, d, rows, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
 }
 
 template <int D, int KIND>

@@ -9,11 +9,32 @@
 
 namespace eattn {
 
+// fp16 operand copies (f16.cu): `count` bf16 tensors of n16 16-byte chunks each; maxbits[t] receives
+// max |x| of tensor t as float bits.
+struct F16Job {
+    const void* src[4];
+    void* dst[4];
+    uint32_t* maxbits;
+    size_t n16;
+    int count;
+};
+cudaError_t launch_to_f16(const F16Job& job, int num_sms, cudaStream_t stream);
+
+// Power-of-two exponent e >= 0 by which a tensor with max |x| = maxbits (float bits) is scaled down in
+// its fp16 copy: 0 while the max is below 2^15, else exponent(max) - 14.
+__host__ __device__ inline int f16_range_exp(uint32_t maxbits) {
+    const int E = (int)((maxbits >> 23) & 0xffu) - 127;
+    return E >= 15 ? E - 14 : 0;
+}
+
 cudaError_t launch_fwd_simt(const FwdArgs& a, bool fp32, cudaStream_t stream);
+cudaError_t launch_fwd_h(const FwdArgs& a, cudaStream_t stream);
+size_t fwd_h_smem_bytes(int nw);
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 size_t fwd_tc_smem_bytes(int d, int nw);
 size_t fwd_simt_smem_bytes(int d, int nkb, int mb, int nw);
 cudaError_t make_tmap_bf16(CUtensorMap* map, const void* base, int BH, int n, int d, int rows);
+cudaError_t make_tmap_f16(CUtensorMap* map, const void* base, int BH, int n, int d, int rows);
 
 // maskT[bh][J][I / 32] bit I % 32 = mask[bh][I][J / 32] bit J % 32
 cudaError_t launch_mask_transpose(const uint32_t* mask, uint32_t* maskT, int BH, int nqb, int nkb, int nw, int nwq,

@@ -131,7 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t sub = kk >> 2, off = (kk & 3) * 32;
-                    mma_bf16_ss(tmem + sb * BN, sdesc_at(kDescK, sQ + sub * (BM * 128) + off),
+                    mma_ss(tmem + sb * BN, sdesc_at(kDescK, sQ + sub * (BM * 128) + off),
                                 sdesc_at(kDescK, kb + sub * (BN * 128) + off), idS, kk > 0);
                 }
                 mma_commit(&bb.s_full[sb]);
@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t vb = sSt + st * C::kStage + C::kBlk;
 #pragma unroll
                 for (int kk = 0; kk < BN / 16; ++kk)
-                    mma_bf16_ss(tmem + C::colO, sdesc_at(kDescK, sP + pb * C::kPBytes + kk * 32),
+                    mma_ss(tmem + C::colO, sdesc_at(kDescK, sP + pb * C::kPBytes + kk * 32),
                                 sdesc_at(kDescMN, vb + kk * 2048), idPV, (J > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(&bb.p_empty[pb]);
                 mma_commit(&bb.kv_empty[st]);

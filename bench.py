@@ -56,7 +56,7 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []  # (monotonic time, csv line)
 
     def __enter__(self):
         try:
@@ -67,11 +67,21 @@ class ClockSampler:
             self.t.start()
         except OSError:
             self.proc = None
+            return self
+        # nvidia-smi takes a moment to start: wait for its first sample so the window is covered
+        t_end = time.monotonic() + 10.0
+        while not self.lines and time.monotonic() < t_end and self.proc.poll() is None:
+            time.sleep(0.02)
+        self.t0 = time.monotonic()
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def stop(self):
+        """Mark the end of the timed region (call right after the closing synchronize)."""
+        self.t1 = time.monotonic()
 
     def __exit__(self, *exc):
         if self.proc:
@@ -84,7 +94,10 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        t0 = getattr(self, "t0", 0.0)
+        t1 = getattr(self, "t1", float("inf"))
+        window = [ln for t, ln in self.lines if t0 - 0.25 <= t <= t1 + 0.25]
+        for ln in window:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -147,7 +160,7 @@ def run_reference(args, rank, world):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
@@ -233,6 +246,7 @@ def main():
             b.entmax_attn_bwd(Q, K, V, O, dO, tau, mask, dQ, dK, dV, ALPHA, True, opts, stream)
             ev[i][2].record(stream)
         torch.cuda.synchronize(dev)
+        clk.stop()
     barrier()
     st = b.entmax_attn_check(stream)
     if st != 0:

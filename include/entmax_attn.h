@@ -69,6 +69,7 @@ typedef struct {
     unsigned long long candidate_blocks; /* pairs the sparse sweeps visited (128-row tiles x 64)  */
     unsigned long long nonzero_blocks;   /* mask bits set                                         */
     unsigned long long sweeps;           /* key sweeps over all tiles (dense + refine + P V)      */
+    unsigned long long overflow_rows;    /* rows whose candidates did not fit the on-chip stash   */
 } entmax_stats;
 
 typedef struct {
