@@ -39,6 +39,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "fwd_common.cuh"
 #include "launch.h"
@@ -79,7 +81,8 @@ enum : int {
     kXCnt1 = 2,              // warpgroup 1: stash count (int bits), -1 when its half overflowed
     kXTau = 3, kXTau2 = 4, kXLo = 5, kXTwo = 6,  // solver state broadcast by warpgroup 0
     kXF0 = 7, kXF1 = 8, kXF2 = 9, kXF0b = 10,    // partial sums of warpgroup 1
-    kXRows = 11
+    kXOvf = 11,                                  // 1: the row's candidates did not fit the stash
+    kXRows = 12
 };
 
 struct Small {
@@ -553,6 +556,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         HistRow h;
         RowSolve s;
         bool row_ovf = false;
+        float Su_stash = 0.f;
         float m_raw = -INFINITY;
         int n1 = 0;
         if (g == 0) {
@@ -572,7 +576,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             solve_init(s, valid ? tau_h : 0.0f, valid ? m : 1.0f, n_i, sp);
             if (!valid) s.done = true;
             if (valid && !row_ovf && a.tau_hist) a.tau_hist[head + row] = tau_h;
-            // rows whose candidates all fit the stash are solved on chip, with no further key sweep
+            // rows whose candidates all fit the stash are solved on chip, with no further key sweep; their
+            // sum of u comes from the stash too (it holds every entry above tau)
             if (ok && valid && !row_ovf) {
                 for (int it = 0; it < kMaxSweeps && !s.done; ++it) {
                     float F0 = 0.f, F1 = 0.f, F2 = 0.f, F0b = 0.f;
@@ -580,7 +585,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     half_sums<KIND>(stash + kHalf * BM, n1, r, sp, s.tau, s.tau2, s.need_two, F0, F1, F2, F0b);
                     solve_step(s, F0, F1, F2, F0b, sp);
                 }
+                float F0 = 0.f, F1 = 0.f, F2 = 0.f, F0b = 0.f;
+                half_sums<KIND>(st_mine, nst, r, sp, s.tau, s.tau, false, F0, F1, F2, F0b);
+                half_sums<KIND>(stash + kHalf * BM, n1, r, sp, s.tau, s.tau, false, F0, F1, F2, F0b);
+                Su_stash = F1;
             }
+            sm.xf[kXOvf][r] = (valid && row_ovf) ? 1.0f : 0.0f;
         }
 
         // ---- histogram sweep for rows whose stash overflowed (warpgroup 0 only) ----
@@ -711,6 +721,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             publish(kSweepPV);
             const float t = sm.xf[kXTau][r], lo0 = sm.xf[kXLo][r];
+            const bool need_sums = __any_sync(0xffffffffu, sm.xf[kXOvf][r] != 0.0f);
             float Sp = 0.f, Sq = 0.f, F2 = 0.f;
             const uint32_t* bits_p = plan_bits + (sw & 1) * W;
             int p = 0;
@@ -725,73 +736,64 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float amax = group_max();
                     const bool keep = sp.cz * amax > lo0;
                     const bool nz = sp.cz * amax - t > 0.f;
-                    // two passes over the block, P then U, through one 32-word array; the sums ride on
-                    // the P pass
+                    // two branch-free passes over the block, P then U, through one 32-word array; the solver
+                    // sums ride on the P pass, in warps that hold a row whose tau still needs the check
                     uint32_t w32[32];
+                    auto p_pass = [&](auto with_sums) {
+                        constexpr bool SUMS = decltype(with_sums)::value;
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        if (sp.cz * gm[q] - t > 0.f) {
+                        for (int c = 0; c < BN; c += 2) {
+                            float p2[2];
 #pragma unroll
-                            for (int e = 0; e < 8; e += 2) {
-                                float p2[2];
-#pragma unroll
-                                for (int c = 0; c < 2; ++c) {
-                                    const float x = sp.cz * vbuf[8 * q + e + c] - t;
-                                    float pp, uu;
-                                    if constexpr (KIND == kAlpha15) {
-                                        uu = fmaxf(x, 0.f);
-                                        pp = uu * uu;
-                                        F2 += x > 0.f ? 1.f : 0.f;
-                                    } else if constexpr (KIND == kAlpha2) {
-                                        pp = fmaxf(x, 0.f);
-                                        uu = x > 0.f ? 1.f : 0.f;
-                                    } else {
-                                        const bool pos = x > 0.f;
-                                        const float xs = pos ? x : 1.f;
-                                        const float u1 = exp2f((sp.k - 1.f) * __log2f(xs));
-                                        uu = pos ? u1 : 0.f;
-                                        pp = uu * xs;
-                                        F2 += pos ? __fdividef(u1, xs) : 0.f;
-                                    }
+                            for (int h2 = 0; h2 < 2; ++h2) {
+                                const float x = sp.cz * vbuf[c + h2] - t;
+                                float pp, uu;
+                                if constexpr (KIND == kAlpha15) {
+                                    uu = fmaxf(x, 0.f);
+                                    pp = uu * uu;
+                                    if constexpr (SUMS) F2 += x > 0.f ? 1.f : 0.f;
+                                } else if constexpr (KIND == kAlpha2) {
+                                    pp = fmaxf(x, 0.f);
+                                    uu = x > 0.f ? 1.f : 0.f;
+                                } else {
+                                    const bool pos = x > 0.f;
+                                    const float xs = pos ? x : 1.f;
+                                    const float u1 = exp2f((sp.k - 1.f) * __log2f(xs));
+                                    uu = pos ? u1 : 0.f;
+                                    pp = uu * xs;
+                                    if constexpr (SUMS) F2 += pos ? __fdividef(u1, xs) : 0.f;
+                                }
+                                if constexpr (SUMS) {
                                     Sp += pp;
                                     Sq += uu;
-                                    p2[c] = pp;
                                 }
-                                w32[4 * q + e / 2] = pack_half2(p2[0], p2[1]);
+                                p2[h2] = pp;
                             }
-                        } else {
-#pragma unroll
-                            for (int w = 4 * q; w < 4 * q + 4; ++w) w32[w] = 0u;
+                            w32[c / 2] = pack_half2(p2[0], p2[1]);
                         }
-                    }
+                    };
+                    if (need_sums) p_pass(std::true_type{});
+                    else p_pass(std::false_type{});
                     // P and U go into the columns of the S tile just read (this warpgroup's own buffer)
                     const uint32_t tp = lane_base + colS;
                     tmem_st32(tp, w32);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        if (sp.cz * gm[q] - t > 0.f) {
+                    for (int c = 0; c < BN; c += 2) {
+                        float u2[2];
 #pragma unroll
-                            for (int e = 0; e < 8; e += 2) {
-                                float u2[2];
-#pragma unroll
-                                for (int c = 0; c < 2; ++c) {
-                                    const float x = sp.cz * vbuf[8 * q + e + c] - t;
-                                    if constexpr (KIND == kAlpha15) {
-                                        u2[c] = fmaxf(x, 0.f);
-                                    } else if constexpr (KIND == kAlpha2) {
-                                        u2[c] = x > 0.f ? 1.f : 0.f;
-                                    } else {
-                                        const bool pos = x > 0.f;
-                                        const float xs = pos ? x : 1.f;
-                                        u2[c] = pos ? exp2f((sp.k - 1.f) * __log2f(xs)) : 0.f;
-                                    }
-                                }
-                                w32[4 * q + e / 2] = pack_half2(u2[0], u2[1]);
+                        for (int h2 = 0; h2 < 2; ++h2) {
+                            const float x = sp.cz * vbuf[c + h2] - t;
+                            if constexpr (KIND == kAlpha15) {
+                                u2[h2] = fmaxf(x, 0.f);
+                            } else if constexpr (KIND == kAlpha2) {
+                                u2[h2] = x > 0.f ? 1.f : 0.f;
+                            } else {
+                                const bool pos = x > 0.f;
+                                const float xs = pos ? x : 1.f;
+                                u2[h2] = pos ? exp2f((sp.k - 1.f) * __log2f(xs)) : 0.f;
                             }
-                        } else {
-#pragma unroll
-                            for (int w = 4 * q; w < 4 * q + 4; ++w) w32[w] = 0u;
                         }
+                        w32[c / 2] = pack_half2(u2[0], u2[1]);
                     }
                     tmem_st32(tp + 32, w32);
                     tmem_st_wait();
@@ -816,12 +818,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = !bar_or256(!ok || *abort_flag != 0);
             bool changed = false;
             if (g == 0) {
-                Sp += sm.xf[kXF0][r];
-                Su = Sq + sm.xf[kXF1][r];
-                F2 += sm.xf[kXF2][r];
-                const float before = s.tau;
-                solve_step(s, Sp, Su, F2, 0.f, sp);
-                changed = s.tau != before;
+                if (row_ovf) {
+                    Sp += sm.xf[kXF0][r];
+                    Su = Sq + sm.xf[kXF1][r];
+                    F2 += sm.xf[kXF2][r];
+                    const float before = s.tau;
+                    solve_step(s, Sp, Su, F2, 0.f, sp);
+                    changed = s.tau != before;
+                } else {
+                    Su = Su_stash;
+                }
             }
             return ok && bar_or256(changed);
         };
