@@ -295,7 +295,22 @@ entmax_status bwd_common(const void* Q, const void* K, const void* V, const void
         a.k = sp.k;
         a.kind = alpha == 1.5f ? kAlpha15 : (alpha == 2.0f ? kAlpha2 : kGeneric);
     }
-    return from_cuda(launch_bwd(a, ws.delta_pad, ws.stat_pad, static_cast<cudaStream_t>(stream)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (!softmax && use_f16_path(d, alpha)) {
+        // fp16 path: the forward left fp16 copies of Q, K, V and their range exponents in the workspace
+        F16Job job;
+        memset(&job, 0, sizeof(job));
+        job.src[0] = dO;
+        job.dst[0] = ws.dOh;
+        job.maxbits = ws.maxbits + 3;
+        job.n16 = (size_t)B * H * n * d / 8;
+        job.count = 1;
+        a.Qh = ws.Qh; a.Kh = ws.Kh; a.Vh = ws.Vh; a.dOh = ws.dOh; a.maxbits = ws.maxbits;
+        cudaError_t e = launch_to_f16(job, num_sms(), s);
+        if (e == cudaSuccess) e = launch_bwd_h(a, ws.delta_pad, ws.stat_pad, s);
+        return from_cuda(e);
+    }
+    return from_cuda(launch_bwd(a, ws.delta_pad, ws.stat_pad, s));
 }
 
 }  // namespace

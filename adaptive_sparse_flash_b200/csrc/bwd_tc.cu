@@ -782,6 +782,14 @@ cudaError_t launch_d(const BwdArgs& a, float* dp, float* sp, cudaStream_t s) {
 
 }  // namespace
 
+cudaError_t launch_bwd_pre(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaStream_t stream) {
+    const int warps = 8;
+    dim3 grid((a.nqb * TB + warps - 1) / warps, a.B * a.H);
+    if (a.d == 64) bwd_pre_kernel<64><<<grid, warps * 32, 0, stream>>>(a, delta_pad, stat_pad);
+    else bwd_pre_kernel<128><<<grid, warps * 32, 0, stream>>>(a, delta_pad, stat_pad);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_bwd(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaStream_t stream) {
     if (a.d == 64) return launch_d<64>(a, delta_pad, stat_pad, stream);
     return launch_d<128>(a, delta_pad, stat_pad, stream);

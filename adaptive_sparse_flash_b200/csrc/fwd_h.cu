@@ -12,15 +12,17 @@
 //   warp 9          TMA issue (one thread): K blocks of 64 keys and, in P V sweeps, V blocks.
 //
 // With A in TMEM an MMA reads only its B operand (2 KB) from shared memory, which keeps shared-memory
-// bandwidth for the K and V tiles. P and U lie in [0, 1] for alpha <= 2, so a single fp16 term each
-// carries 11 significant bits (bf16 would need a two-term split), and P, U of a 64-key block fit the 64
-// columns of its S tile. A new S tile goes into a buffer only after the P V products that read its
+// bandwidth for the K and V tiles. P and U lie in [0, 1] for alpha <= 2. P enters P V as one fp16 term
+// (11 significant bits; bf16 would need a two-term split). U enters as two fp16 terms, U = hi + lo:
+// U V only feeds the backward's delta = dO . (U V) / sum u, which shifts every dS of its row, so it is
+// kept to ~22 bits. P and U hi of a 64-key block fit the 64 columns of its S tile; U lo goes to a
+// buffer of its warpgroup. A new S tile goes into a buffer only after the P V products that read its
 // previous P and U have completed (a commit barrier per buffer), and the MMA thread waits for all P V
 // products at the end of a P V sweep: MMAs into different accumulators are not ordered by issue alone.
 //
-// TMEM columns (512): S buffer b of warpgroup g at 64 (2 g + b), holding P (first 32 columns) and U
+// TMEM columns (512): S buffer b of warpgroup g at 64 (2 g + b), holding P (first 32 columns) and U hi
 // (next 32; K step kk of 16 keys is columns 8 kk .. 8 kk + 7 of each) in P V sweeps; Q at 256 (32
-// columns, 64 fp16 per lane); O at 384, Obar at 448.
+// columns, 64 fp16 per lane); U lo of warpgroup g at 288 + 32 g; O at 384, Obar at 448.
 //
 // Sweeps follow the plan protocol of the bf16 forward (fwd_tc.cu): before each sweep the compute warps
 // publish its kind and its set of key blocks, which the issuing warps follow.
@@ -72,6 +74,7 @@ static_assert(NVS * kKBytes <= kHistBytes, "V ring must fit the histogram region
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColQ = 256;
+constexpr uint32_t kColUlo = 288;
 constexpr uint32_t kColO = 384;
 constexpr uint32_t kColOb = 448;
 
@@ -93,6 +96,7 @@ struct Small {
     uint64_t pv_free[2][2];                // P V products that read a buffer's P and U have completed
     uint64_t pu_full[2][2];                // a buffer's P and U are stored (one barrier per buffer, so
                                            // that no barrier runs two phases ahead of its waiter)
+    uint64_t ulo_free[2];                  // the P V of a warpgroup's last block completed (U lo read)
     uint64_t o_full;
     uint64_t ctrl;
     uint64_t drain[2];
@@ -225,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_init(&sm.pv_free[i][b], 1);
                 mbar_init(&sm.pu_full[i][b], 4);
             }
+            mbar_init(&sm.ulo_free[i], 1);
         }
         mbar_init(&sm.o_full, 1);
         mbar_init(&sm.ctrl, kCompute / 32);
@@ -383,8 +388,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t acc = (tp == 0 && kk == 0) ? 0u : 1u;
                         mma_ts(tmem + kColO, tpu + 8 * kk, dv, idPV, acc);
                         mma_ts(tmem + kColOb, tpu + 32 + 8 * kk, dv, idPV, acc);
+                        mma_ts(tmem + kColOb, tmem + kColUlo + 32u * g + 8 * kk, dv, idPV, 1u);
                     }
                     mma_commit(&sm.pv_free[g][b]);
+                    mma_commit(&sm.ulo_free[g]);
                     mma_commit(&sm.v_empty[vs]);
                     ppar ^= 1u << bi;
                     ++vc;
@@ -777,25 +784,37 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // P and U go into the columns of the S tile just read (this warpgroup's own buffer)
                     const uint32_t tp = lane_base + colS;
                     tmem_st32(tp, w32);
+                    // U = hi + lo: hi next to P, lo into this warpgroup's buffer once the P V of its
+                    // previous block (which read the old lo) completed
+                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.ulo_free[g], (pc & 1) ^ 1, abort_flag, a.status));
+                    if (!ok) break;
 #pragma unroll
-                    for (int c = 0; c < BN; c += 2) {
-                        float u2[2];
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t whi[16], wlo[16];
 #pragma unroll
-                        for (int h2 = 0; h2 < 2; ++h2) {
-                            const float x = sp.cz * vbuf[c + h2] - t;
-                            if constexpr (KIND == kAlpha15) {
-                                u2[h2] = fmaxf(x, 0.f);
-                            } else if constexpr (KIND == kAlpha2) {
-                                u2[h2] = x > 0.f ? 1.f : 0.f;
-                            } else {
-                                const bool pos = x > 0.f;
-                                const float xs = pos ? x : 1.f;
-                                u2[h2] = pos ? exp2f((sp.k - 1.f) * __log2f(xs)) : 0.f;
+                        for (int c = 0; c < 32; c += 2) {
+                            float u2[2];
+#pragma unroll
+                            for (int h2 = 0; h2 < 2; ++h2) {
+                                const float x = sp.cz * vbuf[32 * h + c + h2] - t;
+                                if constexpr (KIND == kAlpha15) {
+                                    u2[h2] = fmaxf(x, 0.f);
+                                } else if constexpr (KIND == kAlpha2) {
+                                    u2[h2] = x > 0.f ? 1.f : 0.f;
+                                } else {
+                                    const bool pos = x > 0.f;
+                                    const float xs = pos ? x : 1.f;
+                                    u2[h2] = pos ? exp2f((sp.k - 1.f) * __log2f(xs)) : 0.f;
+                                }
                             }
+                            const __half2 hh = __floats2half2_rn(u2[0], u2[1]);
+                            const float2 hf = __half22float2(hh);
+                            whi[c / 2] = *reinterpret_cast<const uint32_t*>(&hh);
+                            wlo[c / 2] = pack_half2(u2[0] - hf.x, u2[1] - hf.y);
                         }
-                        w32[c / 2] = pack_half2(u2[0], u2[1]);
+                        tmem_st16(tp + 32 + 16 * h, whi);
+                        tmem_st16(lane_base + kColUlo + 32u * g + 16 * h, wlo);
                     }
-                    tmem_st32(tp + 32, w32);
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();

@@ -63,9 +63,17 @@ struct BwdArgs {
     float cz;               // entmax: (alpha - 1) * scale
     float k;                // entmax: 1 / (alpha - 1)
     int kind;               // entmax AlphaKind
+    // fp16 path (bwd_h.cu): copies of Q, K, V (from the forward) and dO, and their range exponents
+    const void* Qh;
+    const void* Kh;
+    const void* Vh;
+    const void* dOh;
+    const uint32_t* maxbits;  // [4]: Q, K, V, dO
 };
 
 cudaError_t launch_bwd(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaStream_t stream);
+cudaError_t launch_bwd_pre(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaStream_t stream);
+cudaError_t launch_bwd_h(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaStream_t stream);
 size_t bwd_smem_bytes(int d, int nw, int nwq);
 
 struct SoftmaxFwdArgs {
