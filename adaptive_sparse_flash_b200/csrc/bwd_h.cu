@@ -104,6 +104,12 @@ __device__ __forceinline__ void split_half2(float a, float b, uint32_t& hi, uint
     lo = pack_half2(a - hf.x, b - hf.y);
 }
 
+__device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
 struct Bars {
     uint64_t tile_full;
     uint64_t q_full[NST], q_empty[NST];
@@ -325,22 +331,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(lane_base + 128u * g, reinterpret_cast<uint32_t*>(sv));
                 tmem_ld32(lane_base + 128u * g + 32, reinterpret_cast<uint32_t*>(sv) + 32);
                 tmem_ld_wait();
-                const float* stat = reinterpret_cast<const float*>(smem + kvOffSt + st * kStageKV + 2 * kBlk);
-                const float* dlt = stat + 64;
+                const uint32_t sstat = sSt + st * kStageKV + 2 * kBlk;  // tau[64], then delta[64]
                 const int q0 = I * TB;
                 const bool full = kvalid && (q0 + TB <= a.n) && (!a.causal || q0 >= k0 + TM - 1);
+                // entries outside the causal / valid range get -inf (a partial block is the rare case)
+                if (__any_sync(0xffffffffu, !full)) {
+#pragma unroll
+                    for (int c = 0; c < TB; ++c) {
+                        const int qi = q0 + c;
+                        if (!(kvalid && qi < a.n && (!a.causal || qi >= key))) sv[c] = -INFINITY;
+                    }
+                }
                 // P^T row of this key against the 64 queries of block I; u kept in sv
                 uint32_t w32[32];
 #pragma unroll
                 for (int c = 0; c < TB; c += 4) {
-                    const float4 t4 = *reinterpret_cast<const float4*>(stat + c);
+                    const float4 t4 = ld_shared_f4(sstat + 4 * c);
                     const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
                     float pp[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int qi = q0 + c + e;
-                        const bool okc = full || (kvalid && qi < a.n && (!a.causal || qi >= key));
-                        const float x = okc ? fmaf(sv[c + e], sc.cz, -tv[e]) : -1.f;
+                        const float x = fmaf(sv[c + e], sc.cz, -tv[e]);
                         float u;
                         entmax_pu<KIND>(x, a.k, pp[e], u);
                         sv[c + e] = u;
@@ -363,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t whi[16], wlo[16];
 #pragma unroll
                     for (int c = 0; c < 32; c += 4) {
-                        const float4 d4 = *reinterpret_cast<const float4*>(dlt + 32 * h + c);
+                        const float4 d4 = ld_shared_f4(sstat + 256 + 4 * (32 * h + c));
                         const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
                         float ds[4];
 #pragma unroll
@@ -573,11 +584,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_wait();
                 const int j0 = J * TB;
                 const bool full = qvalid && (j0 + TB <= a.n) && (!a.causal || j0 + TB - 1 <= q0);
+                if (__any_sync(0xffffffffu, !full)) {
+#pragma unroll
+                    for (int c = 0; c < TB; ++c) {
+                        const int kj = j0 + c;
+                        if (!(qvalid && kj < a.n && (!a.causal || kj <= row))) sv[c] = -INFINITY;
+                    }
+                }
 #pragma unroll
                 for (int c = 0; c < TB; ++c) {
-                    const int kj = j0 + c;
-                    const bool okc = full || (qvalid && kj < a.n && (!a.causal || kj <= row));
-                    const float x = okc ? fmaf(sv[c], sc.cz, -tau) : -1.f;
+                    const float x = fmaf(sv[c], sc.cz, -tau);
                     float p, u;
                     entmax_pu<KIND>(x, a.k, p, u);
                     sv[c] = u;
