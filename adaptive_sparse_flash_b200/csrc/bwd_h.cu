@@ -180,8 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                       const BwdArgs a, const float* __restrict__ delta_pad, const float* __restrict__ stat_pad) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~(uintptr_t)1023);
+    unsigned char* smem = align_smem_1024(smem_raw);
     Bars& bb = *reinterpret_cast<Bars*>(smem + kvOffBar);
     uint32_t* vis = reinterpret_cast<uint32_t*>(&bb + 1);  // [nwq] query blocks to visit
 
@@ -445,8 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const BwdArgs a, const float* __restrict__ delta_pad, const float* __restrict__ stat_pad) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~(uintptr_t)1023);
+    unsigned char* smem = align_smem_1024(smem_raw);
     Bars& bb = *reinterpret_cast<Bars*>(smem + qOffBar);
     uint32_t* vis = reinterpret_cast<uint32_t*>(&bb + 1);  // [nw] key blocks to visit
 

@@ -184,8 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const BwdArgs a, const float* __restrict__ delta_pad, const float* __restrict__ stat_pad) {
     using C = CfgKV<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~(uintptr_t)1023);
+    unsigned char* smem = align_smem_1024(smem_raw);
     BarsKV& bb = *reinterpret_cast<BarsKV*>(smem + C::offBar);
     uint32_t* vis = reinterpret_cast<uint32_t*>(&bb + 1);  // [nwq] query blocks to visit
 
@@ -491,8 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const BwdArgs a, const float* __restrict__ delta_pad, const float* __restrict__ stat_pad) {
     using C = CfgQ<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~(uintptr_t)1023);
+    unsigned char* smem = align_smem_1024(smem_raw);
     BarsKV& bb = *reinterpret_cast<BarsKV*>(smem + C::offBar);
     uint32_t* vis = reinterpret_cast<uint32_t*>(&bb + 1);  // [nw] key blocks to visit
 

@@ -22,6 +22,13 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared-memory base rounded up to 1024 bytes (the 128B-swizzled tiles need it). Pointer
+// arithmetic on the shared array itself, not a round trip through an integer, so that the compiler
+// still knows the result points to shared memory and emits shared (not generic) loads and stores.
+__device__ __forceinline__ unsigned char* align_smem_1024(unsigned char* base) {
+    return base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -4,25 +4,23 @@
 // One CTA per (b, h, 128-row query tile), 352 threads:
 //   warps 0-3, 4-7  compute warpgroups 0 and 1. Thread r of a warpgroup owns query row r of the tile
 //                   and reads TMEM lane r; the two warpgroups take alternate key blocks of every sweep;
-//   warp 8          S issue (one thread): S = Q K^T with the Q tile held in TMEM (A operand from tensor
-//                   memory), into two TMEM buffers per warpgroup;
+//   warp 8          S issue (one thread): S = Q K^T from shared memory into two TMEM buffers per
+//                   warpgroup;
 //   warp 10         P V issue (one thread): O += P V and Obar += U V with P and U stored by the compute
 //                   warps into the TMEM columns of the S tile they came from. Two issuing threads keep the
 //                   tensor pipe fed: each waits only on its own barriers, in block order;
-//   warp 9          TMA issue (one thread): K blocks of 64 keys and, in P V sweeps, V blocks.
+//   warp 9          TMA issue (one thread): Q once, K blocks of 64 keys and, in P V sweeps, V blocks.
 //
-// With A in TMEM an MMA reads only its B operand (2 KB) from shared memory, which keeps shared-memory
-// bandwidth for the K and V tiles. P and U lie in [0, 1] for alpha <= 2. P enters P V as one fp16 term
-// (11 significant bits; bf16 would need a two-term split). U enters as two fp16 terms, U = hi + lo:
-// U V only feeds the backward's delta = dO . (U V) / sum u, which shifts every dS of its row, so it is
-// kept to ~22 bits. P and U hi of a 64-key block fit the 64 columns of its S tile; U lo goes to a
-// buffer of its warpgroup. A new S tile goes into a buffer only after the P V products that read its
+// P and U lie in [0, 1] for alpha <= 2. P enters P V as one fp16 term (11 significant bits; bf16 would
+// need a two-term split). U enters as two fp16 terms, U = hi + lo: U V only feeds the backward's
+// delta = dO . (U V) / sum u, which shifts every dS of its row, so it is kept to ~22 bits. P and U hi
+// of a 64-key block fit the 64 columns of its S tile; U lo goes to a 32-column buffer paired with it. A new S tile goes into a buffer only after the P V products that read its
 // previous P and U have completed (a commit barrier per buffer), and the MMA thread waits for all P V
 // products at the end of a P V sweep: MMAs into different accumulators are not ordered by issue alone.
 //
 // TMEM columns (512): S buffer b of warpgroup g at 64 (2 g + b), holding P (first 32 columns) and U hi
-// (next 32; K step kk of 16 keys is columns 8 kk .. 8 kk + 7 of each) in P V sweeps; Q at 256 (32
-// columns, 64 fp16 per lane); U lo of warpgroup g at 288 + 32 g; O at 384, Obar at 448.
+// (next 32; K step kk of 16 keys is columns 8 kk .. 8 kk + 7 of each) in P V sweeps; the U lo of that
+// buffer at 256 + 32 (2 g + b); O at 384, Obar at 448.
 //
 // Sweeps follow the plan protocol of the bf16 forward (fwd_tc.cu): before each sweep the compute warps
 // publish its kind and its set of key blocks, which the issuing warps follow.
@@ -57,7 +55,7 @@ constexpr int kThreads = 352;
 constexpr int kCompute = 256;
 constexpr int NKS = 4;
 constexpr int NVS = 8;
-constexpr int kHalf = 96;  // stash entries per row and warpgroup
+constexpr int kHalf = 88;  // stash entries per row and warpgroup
 
 constexpr uint64_t kDescK = sdesc_sw128_fields(16, 1024);
 constexpr uint64_t kDescMN = sdesc_sw128_fields(64 * 128, 1024);
@@ -65,7 +63,9 @@ constexpr uint64_t kDescMN = sdesc_sw128_fields(64 * 128, 1024);
 constexpr uint32_t kKBytes = BN * D * 2;                 // 8 KB per K or V block
 constexpr uint32_t kHistBytes = 256u * BM * 2u;          // u16 [256][128]
 constexpr uint32_t kStashBytes = 2u * kHalf * BM * 4u;   // fp32 [2][kHalf][128]
-constexpr uint32_t offK = 0;
+constexpr uint32_t kQBytes = BM * D * 2;                 // 16 KB
+constexpr uint32_t offQ = 0;
+constexpr uint32_t offK = offQ + kQBytes;
 constexpr uint32_t offHist = offK + NKS * kKBytes;
 constexpr uint32_t offStash = offHist + kHistBytes;
 constexpr uint32_t offV = offHist;  // the V ring reuses the histogram (dead in P V sweeps)
@@ -73,8 +73,7 @@ constexpr uint32_t offSmall = offStash + kStashBytes;
 static_assert(NVS * kKBytes <= kHistBytes, "V ring must fit the histogram region");
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColQ = 256;
-constexpr uint32_t kColUlo = 288;
+constexpr uint32_t kColUlo = 256;
 constexpr uint32_t kColO = 384;
 constexpr uint32_t kColOb = 448;
 
@@ -89,14 +88,13 @@ enum : int {
 };
 
 struct Small {
-    uint64_t q_ready;
+    uint64_t q_full;
     uint64_t k_full[NKS], k_empty[NKS];
     uint64_t v_full[NVS], v_empty[NVS];
     uint64_t s_full[2][2], s_empty[2][2];  // [warpgroup][buffer]
     uint64_t pv_free[2][2];                // P V products that read a buffer's P and U have completed
     uint64_t pu_full[2][2];                // a buffer's P and U are stored (one barrier per buffer, so
                                            // that no barrier runs two phases ahead of its waiter)
-    uint64_t ulo_free[2];                  // the P V of a warpgroup's last block completed (U lo read)
     uint64_t o_full;
     uint64_t ctrl;
     uint64_t drain[2];
@@ -195,10 +193,10 @@ __device__ __forceinline__ bool block_full(int J, int n, int causal, int row0) {
 
 template <int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
-    fwd_h_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+    fwd_h_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~(uintptr_t)1023);
+    unsigned char* smem = align_smem_1024(smem_raw);
     Small& sm = *reinterpret_cast<Small*>(smem + offSmall);
     const int W = a.nw;
     uint32_t* plan_bits = reinterpret_cast<uint32_t*>(&sm + 1);  // [2][W]
@@ -219,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &sm.abort_flag;
 
     if (tid == 0) {
-        mbar_init(&sm.q_ready, 4);
+        mbar_init(&sm.q_full, 1);
         for (int i = 0; i < NKS; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
         for (int i = 0; i < NVS; ++i) { mbar_init(&sm.v_full[i], 1); mbar_init(&sm.v_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
@@ -229,7 +227,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_init(&sm.pv_free[i][b], 1);
                 mbar_init(&sm.pu_full[i][b], 4);
             }
-            mbar_init(&sm.ulo_free[i], 1);
         }
         mbar_init(&sm.o_full, 1);
         mbar_init(&sm.ctrl, kCompute / 32);
@@ -247,14 +244,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    const uint32_t sQ = smem_u32(smem + offQ);
     const uint32_t sK0 = smem_u32(smem + offK);
     const uint32_t sV0 = smem_u32(smem + offV);
 
     if (warp == 9) {
         // ------------------------------------------------------------------ TMA issue
         if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
+            mbar_arrive_expect_tx(&sm.q_full, kQBytes);
+            tma_load_3d(smem + offQ, &tmQ, &sm.q_full, 0, row0, bh);
             uint32_t lc = 0, vc = 0;
             bool ok = true;
             for (int sw = 0; ok; ++sw) {
@@ -287,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     wait_drain(&sm.k_full[i % NKS], (i / NKS) & 1, 100000000ull);
                 for (uint32_t i = (vc > (uint32_t)NVS ? vc - NVS : 0); i < vc; ++i)
                     wait_drain(&sm.v_full[i % NVS], (i / NVS) & 1, 100000000ull);
+                wait_drain(&sm.q_full, 0, 100000000ull);
             }
         }
     } else if (warp == 8) {
@@ -300,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t ppar = 0xfu;
             bool after_pv = false;
             int npv = 0;
-            bool ok = wait_bounded(&sm.q_ready, 0, abort_flag, a.status, true);
+            bool ok = wait_bounded(&sm.q_full, 0, abort_flag, a.status, true);
             tc_fence_after();
             for (int sw = 0; ok; ++sw) {
                 if (!(ok = wait_bounded(&sm.ctrl, sw & 1, abort_flag, a.status, true))) break;
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t dS = tmem + 64u * bi;
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk)
-                        mma_ts(dS, tmem + kColQ + 8 * kk, sdesc_at(kDescK, kbase + kk * 32), idS, kk > 0 ? 1u : 0u);
+                        mma_ss(dS, sdesc_at(kDescK, sQ + kk * 32), sdesc_at(kDescK, kbase + kk * 32), idS, kk > 0 ? 1u : 0u);
                     mma_commit(&sm.s_full[g][b]);
                     mma_commit(&sm.k_empty[ks]);
                     ++lc;
@@ -388,10 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t acc = (tp == 0 && kk == 0) ? 0u : 1u;
                         mma_ts(tmem + kColO, tpu + 8 * kk, dv, idPV, acc);
                         mma_ts(tmem + kColOb, tpu + 32 + 8 * kk, dv, idPV, acc);
-                        mma_ts(tmem + kColOb, tmem + kColUlo + 32u * g + 8 * kk, dv, idPV, 1u);
+                        mma_ts(tmem + kColOb, tmem + kColUlo + 32u * bi + 8 * kk, dv, idPV, 1u);
                     }
                     mma_commit(&sm.pv_free[g][b]);
-                    mma_commit(&sm.ulo_free[g]);
                     mma_commit(&sm.v_empty[vs]);
                     ppar ^= 1u << bi;
                     ++vc;
@@ -435,22 +436,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         sm.xf[kXMax0 + g][r] = -INFINITY;
         if (tid == 0) sm.plan_kind[0] = kSweepDense;
 
-        // Q tile into TMEM (warpgroup 0): row r's 64 fp16 as 32 columns of lane r
-        if (g == 0) {
-            uint32_t qv[32];
-            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const __half*>(a.Qh) +
-                                                              (head + (size_t)(valid ? row : 0)) * D);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const uint4 x = valid ? src[i] : make_uint4(0u, 0u, 0u, 0u);
-                qv[4 * i] = x.x; qv[4 * i + 1] = x.y; qv[4 * i + 2] = x.z; qv[4 * i + 3] = x.w;
-            }
-            tmem_st32(lane_base + kColQ, qv);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.q_ready);
-        }
         named_bar_sync(1, kCompute);
         if (lane == 0) mbar_arrive(&sm.ctrl);
 
@@ -784,10 +769,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // P and U go into the columns of the S tile just read (this warpgroup's own buffer)
                     const uint32_t tp = lane_base + colS;
                     tmem_st32(tp, w32);
-                    // U = hi + lo: hi next to P, lo into this warpgroup's buffer once the P V of its
-                    // previous block (which read the old lo) completed
-                    ok = __all_sync(0xffffffffu, wait_bounded(&sm.ulo_free[g], (pc & 1) ^ 1, abort_flag, a.status));
-                    if (!ok) break;
+                    // U = hi + lo: hi next to P, lo into the buffer paired with this S buffer (free for the
+                    // same reason: this S tile was issued after the P V that read the old contents)
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         uint32_t whi[16], wlo[16];
@@ -813,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             wlo[c / 2] = pack_half2(u2[0] - hf.x, u2[1] - hf.y);
                         }
                         tmem_st16(tp + 32 + 16 * h, whi);
-                        tmem_st16(lane_base + kColUlo + 32u * g + 16 * h, wlo);
+                        tmem_st16(lane_base + kColUlo + (colS >> 1) + 16 * h, wlo);
                     }
                     tmem_st_wait();
                     tc_fence_before();
@@ -946,8 +929,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int KIND>
 cudaError_t launch_fwd_h_t(const FwdArgs& a, cudaStream_t stream) {
-    CUtensorMap tk, tv;
+    CUtensorMap tq, tk, tv;
     cudaError_t e;
+    if ((e = make_tmap_f16(&tq, a.Qh, a.B * a.H, a.n, D, BM)) != cudaSuccess) return e;
     if ((e = make_tmap_f16(&tk, a.Kh, a.B * a.H, a.n, D, BN)) != cudaSuccess) return e;
     if ((e = make_tmap_f16(&tv, a.Vh, a.B * a.H, a.n, D, BN)) != cudaSuccess) return e;
     const size_t bytes = fwd_h_smem_bytes(a.nw);
@@ -956,7 +940,7 @@ cudaError_t launch_fwd_h_t(const FwdArgs& a, cudaStream_t stream) {
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
         return e;
     dim3 grid(a.ntiles, a.B * a.H);
-    kern<<<grid, kThreads, bytes, stream>>>(tk, tv, a);
+    kern<<<grid, kThreads, bytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError();
 }
 

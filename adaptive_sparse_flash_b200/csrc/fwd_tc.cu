@@ -149,8 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     using C = Cfg<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     // 1024-byte alignment for the 128B-swizzled tiles
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~(uintptr_t)1023);
+    unsigned char* smem = align_smem_1024(smem_raw);
     Small& sm = *reinterpret_cast<Small*>(smem + C::offSmall);
     const int W = a.nw;
     uint32_t* plan_bits = reinterpret_cast<uint32_t*>(&sm + 1);  // [2][W]

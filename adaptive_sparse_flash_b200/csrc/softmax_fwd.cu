@@ -56,8 +56,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        const __grid_constant__ CUtensorMap tmV, const SoftmaxFwdArgs a) {
     using C = CfgS<D>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
-    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                                           ~(uintptr_t)1023);
+    unsigned char* smem = align_smem_1024(smem_raw);
     BarsS& bb = *reinterpret_cast<BarsS*>(smem + C::offBar);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qt = a.ntiles - 1 - (int)blockIdx.x;
