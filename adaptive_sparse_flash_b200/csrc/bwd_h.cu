@@ -25,11 +25,14 @@
 //   bwd_h_dkdv  one CTA per 128-key tile, walking the query blocks of the transposed mask:
 //               S^T = K Q^T, dP^T = V dO^T; dV += P^T dO, dK += dS^T Q.
 //               TMEM: S^T / dP^T of warpgroup g at 128 g / 128 g + 64 (P^T overwrites the first 32
-//               columns of S^T), [dS^T hi | dS^T lo] of g at 256 + 64 g, dV at 384, dK at 448. A new S^T
-//               goes into a buffer only after the gradient MMAs that read its P^T completed.
+//               columns of S^T), [dS^T hi | dS^T lo] of g at 256 + 64 g, dV at 384, dK at 448. The dV
+//               products of a block go as soon as its P^T is stored and run one block ahead of the dK
+//               products; a new S^T goes into a buffer once the dV products that read its P^T completed.
 //   bwd_h_dq    one CTA per 128-row query tile, walking the key blocks of the row mask:
 //               S = Q K^T, dP = dO V^T; dQ += dS K.
 //               TMEM: S / dP of g at 128 g / 128 g + 64, [dS hi | dS lo] of g at 256 + 64 g, dQ at 384.
+// Score and dP tiles have their own full / empty barriers and are released as soon as the warpgroup has
+// read them, so the next block's products can run while the warpgroup still computes.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -113,8 +116,10 @@ __device__ __forceinline__ float4 ld_shared_f4(uint32_t addr) {
 struct Bars {
     uint64_t tile_full;
     uint64_t q_full[NST], q_empty[NST];
-    uint64_t s_full[2], s_empty[2];
-    uint64_t a_full[2], a_empty[2];
+    uint64_t s_full[2], s_empty[2];  // score tile: MMA done / buffer free again
+    uint64_t d_full[2], d_empty[2];  // dP tile: MMA done / read by the warpgroup
+    uint64_t p_full[2], p_empty[2];  // dK / dV: P^T stored / the dV MMAs that read it done
+    uint64_t a_full[2], a_empty[2];  // dS operands stored / the MMAs that read them done
     uint64_t acc_full;
     uint64_t drain[2];
     uint32_t tmem_base;
@@ -156,6 +161,10 @@ __device__ __forceinline__ void init_bars(Bars& bb) {
     for (int i = 0; i < 2; ++i) {
         mbar_init(&bb.s_full[i], 1);
         mbar_init(&bb.s_empty[i], 4);
+        mbar_init(&bb.d_full[i], 1);
+        mbar_init(&bb.d_empty[i], 4);
+        mbar_init(&bb.p_full[i], 4);
+        mbar_init(&bb.p_empty[i], 1);
         mbar_init(&bb.a_full[i], 4);
         mbar_init(&bb.a_empty[i], 1);
     }
@@ -255,39 +264,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int g = t & 1;
                 const uint32_t j = (uint32_t)(t >> 1), st = (uint32_t)t % NST;
                 if (!(ok = wait_bounded(&bb.q_full[st], ((uint32_t)t / NST) & 1, abort_flag, a.status, true))) break;
-                if (!(ok = wait_bounded(&bb.s_empty[g], (j & 1) ^ 1, abort_flag, a.status, true))) break;
-                // P^T of the warpgroup's previous block lives in this S^T buffer: its gradient MMAs first
-                if (!(ok = wait_bounded(&bb.a_empty[g], (j & 1) ^ 1, abort_flag, a.status, true))) break;
+                // S^T buffer: the warpgroup's previous P^T (written over its S^T) read by the dV MMAs
+                if (!(ok = wait_bounded(&bb.p_empty[g], (j & 1) ^ 1, abort_flag, a.status, true))) break;
                 tc_fence_after();
                 const uint32_t qb = sSt + st * kStageKV, ob = qb + kBlk;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + 128u * g, sdesc_at(kDescK, sK + kk * 32), sdesc_at(kDescK, qb + kk * 32), idS, kk > 0);
+                mma_commit(&bb.s_full[g]);
+                // dP^T buffer: read by the warpgroup for its previous block
+                if (!(ok = wait_bounded(&bb.d_empty[g], (j & 1) ^ 1, abort_flag, a.status, true))) break;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + 128u * g + 64, sdesc_at(kDescK, sV + kk * 32), sdesc_at(kDescK, ob + kk * 32), idS,
                            kk > 0);
-                mma_commit(&bb.s_full[g]);
+                mma_commit(&bb.d_full[g]);
             }
             mma_commit(&bb.drain[0]);
             wait_drain(&bb.drain[0], 0, 200000000ull);
         }
     } else if (warp == 10) {
         // ------------------------------------------------------------------ gradient issue
+        // dV of a block as soon as its P^T is stored (that frees the S^T buffer for the next block), dK
+        // once its dS^T is: the dV products run one block ahead of the dK products.
         if (lane == 0) {
             constexpr uint32_t idG = idesc_f16_f32(TM, D, false, true);  // P^T dO, dS^T Q (MN-major B)
             bool ok = true;
-            for (int t = 0; t < T && ok; ++t) {
+            auto issue_dv = [&](int t) -> bool {
                 const int g = t & 1;
                 const uint32_t j = (uint32_t)(t >> 1), st = (uint32_t)t % NST;
-                if (!(ok = wait_bounded(&bb.a_full[g], j & 1, abort_flag, a.status, true))) break;
+                if (!wait_bounded(&bb.p_full[g], j & 1, abort_flag, a.status, true)) return false;
                 tc_fence_after();
-                const uint32_t qb = sSt + st * kStageKV, ob = qb + kBlk;
-                const uint32_t tpt = tmem + 128u * g;        // P^T
-                const uint32_t ta = tmem + 256u + 64u * g;   // dS^T hi, lo
+                const uint32_t ob = sSt + st * kStageKV + kBlk;
+                const uint32_t tpt = tmem + 128u * g;  // P^T
 #pragma unroll
                 for (int kk = 0; kk < TB / 16; ++kk)
                     mma_ts(tmem + 384, tpt + 8 * kk, sdesc_at(kDescMN, ob + kk * 2048), idG, (t == 0 && kk == 0) ? 0u : 1u);
+                mma_commit(&bb.p_empty[g]);
+                return true;
+            };
+            auto issue_dk = [&](int t) -> bool {
+                const int g = t & 1;
+                const uint32_t j = (uint32_t)(t >> 1), st = (uint32_t)t % NST;
+                if (!wait_bounded(&bb.a_full[g], j & 1, abort_flag, a.status, true)) return false;
+                tc_fence_after();
+                const uint32_t qb = sSt + st * kStageKV;
+                const uint32_t ta = tmem + 256u + 64u * g;  // dS^T hi, lo
 #pragma unroll
                 for (int kk = 0; kk < TB / 16; ++kk) {
                     const uint64_t dq = sdesc_at(kDescMN, qb + kk * 2048);
@@ -295,8 +318,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_ts(tmem + 448, ta + 32 + 8 * kk, dq, idG, 1u);
                 }
                 mma_commit(&bb.a_empty[g]);
-                mma_commit(&bb.q_empty[st]);
+                mma_commit(&bb.q_empty[st]);  // after the block's dV and dK (and its score MMAs)
+                return true;
+            };
+            for (int t = 0; t < T && ok; ++t) {
+                ok = issue_dv(t);
+                if (ok && t > 0) ok = issue_dk(t - 1);
             }
+            if (ok && T > 0) ok = issue_dk(T - 1);
             if (ok && T > 0) mma_commit(&bb.acc_full);
             mma_commit(&bb.drain[1]);
             wait_drain(&bb.drain[1], 0, 200000000ull);
@@ -341,57 +370,65 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!(kvalid && qi < a.n && (!a.causal || qi >= key))) sv[c] = -INFINITY;
                     }
                 }
-                // P^T row of this key against the 64 queries of block I; u kept in sv
-                uint32_t w32[32];
+                // P^T row of this key against the 64 queries of block I, written over its S^T; u kept in sv
+                {
+                    uint32_t w32[32];
+#pragma unroll
+                    for (int c = 0; c < TB; c += 4) {
+                        const float4 t4 = ld_shared_f4(sstat + 4 * c);
+                        const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
+                        float pp[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float x = fmaf(sv[c + e], sc.cz, -tv[e]);
+                            float u;
+                            entmax_pu<KIND>(x, a.k, pp[e], u);
+                            sv[c + e] = u;
+                        }
+                        w32[c / 2] = pack_half2(pp[0], pp[1]);
+                        w32[c / 2 + 1] = pack_half2(pp[2], pp[3]);
+                    }
+                    tmem_st32(lane_base + 128u * g, w32);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bb.p_full[g]);
+                // dS^T = u (dP^T - delta), formed in place of dP^T
+                ok = __all_sync(0xffffffffu, wait_bounded(&bb.d_full[g], j & 1, abort_flag, a.status));
+                if (!ok) break;
+                tc_fence_after();
+                __syncwarp();
+                float dp[TB];
+                tmem_ld32(lane_base + 128u * g + 64, reinterpret_cast<uint32_t*>(dp));
+                tmem_ld32(lane_base + 128u * g + 96, reinterpret_cast<uint32_t*>(dp) + 32);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bb.d_empty[g]);
 #pragma unroll
                 for (int c = 0; c < TB; c += 4) {
-                    const float4 t4 = ld_shared_f4(sstat + 4 * c);
-                    const float tv[4] = {t4.x, t4.y, t4.z, t4.w};
-                    float pp[4];
+                    const float4 d4 = ld_shared_f4(sstat + 256 + 4 * c);
+                    const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float x = fmaf(sv[c + e], sc.cz, -tv[e]);
-                        float u;
-                        entmax_pu<KIND>(x, a.k, pp[e], u);
-                        sv[c + e] = u;
-                    }
-                    w32[c / 2] = pack_half2(pp[0], pp[1]);
-                    w32[c / 2 + 1] = pack_half2(pp[2], pp[3]);
+                    for (int e = 0; e < 4; ++e) dp[c + e] = sv[c + e] * (dp[c + e] - dv4[e] * sc.dl) * sc.ds;
                 }
-                // P^T over the S^T just read (the score thread issued this S^T after the previous gradient
-                // MMAs of this warpgroup completed); the dS^T buffer is free once they did
-                tmem_st32(lane_base + 128u * g, w32);
+                // the dS^T buffer is free once this warpgroup's previous dK MMAs completed
                 ok = __all_sync(0xffffffffu, wait_bounded(&bb.a_empty[g], (j & 1) ^ 1, abort_flag, a.status));
                 if (!ok) break;
                 const uint32_t ta = lane_base + 256u + 64u * g;
-                // dS^T = u (dP^T - delta), in two halves of 32 queries
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    float dp[32];
-                    tmem_ld32(lane_base + 128u * g + 64 + 32 * h, reinterpret_cast<uint32_t*>(dp));
-                    tmem_ld_wait();
                     uint32_t whi[16], wlo[16];
 #pragma unroll
-                    for (int c = 0; c < 32; c += 4) {
-                        const float4 d4 = ld_shared_f4(sstat + 256 + 4 * (32 * h + c));
-                        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
-                        float ds[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            ds[e] = sv[32 * h + c + e] * (dp[c + e] - dv4[e] * sc.dl) * sc.ds;
-                        split_half2(ds[0], ds[1], whi[c / 2], wlo[c / 2]);
-                        split_half2(ds[2], ds[3], whi[c / 2 + 1], wlo[c / 2 + 1]);
-                    }
+                    for (int c = 0; c < 32; c += 2) split_half2(dp[32 * h + c], dp[32 * h + c + 1], whi[c / 2], wlo[c / 2]);
                     tmem_st16(ta + 16 * h, whi);
                     tmem_st16(ta + 32 + 16 * h, wlo);
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&bb.s_empty[g]);
-                    mbar_arrive(&bb.a_full[g]);
-                }
+                if (lane == 0) mbar_arrive(&bb.a_full[g]);
                 ++j;
             }
         }
@@ -520,11 +557,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + 128u * g, sdesc_at(kDescK, sQ + kk * 32), sdesc_at(kDescK, kb + kk * 32), idS, kk > 0);
+                mma_commit(&bb.s_full[g]);
+                if (!(ok = wait_bounded(&bb.d_empty[g], (j & 1) ^ 1, abort_flag, a.status, true))) break;
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
                     mma_ss(tmem + 128u * g + 64, sdesc_at(kDescK, sO + kk * 32), sdesc_at(kDescK, vb + kk * 32), idS,
                            kk > 0);
-                mma_commit(&bb.s_full[g]);
+                mma_commit(&bb.d_full[g]);
             }
             mma_commit(&bb.drain[0]);
             wait_drain(&bb.drain[0], 0, 200000000ull);
@@ -580,6 +620,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld32(lane_base + 128u * g, reinterpret_cast<uint32_t*>(sv));
                 tmem_ld32(lane_base + 128u * g + 32, reinterpret_cast<uint32_t*>(sv) + 32);
                 tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bb.s_empty[g]);  // the score buffer is free for the next block
                 const int j0 = J * TB;
                 const bool full = qvalid && (j0 + TB <= a.n) && (!a.causal || j0 + TB - 1 <= q0);
                 if (__any_sync(0xffffffffu, !full)) {
@@ -596,29 +639,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                     entmax_pu<KIND>(x, a.k, p, u);
                     sv[c] = u;
                 }
+                ok = __all_sync(0xffffffffu, wait_bounded(&bb.d_full[g], j & 1, abort_flag, a.status));
+                if (!ok) break;
+                tc_fence_after();
+                __syncwarp();
+                float dp[TB];
+                tmem_ld32(lane_base + 128u * g + 64, reinterpret_cast<uint32_t*>(dp));
+                tmem_ld32(lane_base + 128u * g + 96, reinterpret_cast<uint32_t*>(dp) + 32);
+                tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bb.d_empty[g]);
+#pragma unroll
+                for (int c = 0; c < TB; ++c) dp[c] = sv[c] * (dp[c] - dl) * sc.ds;
                 ok = __all_sync(0xffffffffu, wait_bounded(&bb.a_empty[g], (j & 1) ^ 1, abort_flag, a.status));
                 if (!ok) break;
                 const uint32_t ta = lane_base + 256u + 64u * g;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    float dp[32];
-                    tmem_ld32(lane_base + 128u * g + 64 + 32 * h, reinterpret_cast<uint32_t*>(dp));
-                    tmem_ld_wait();
                     uint32_t whi[16], wlo[16];
 #pragma unroll
-                    for (int c = 0; c < 32; c += 2)
-                        split_half2(sv[32 * h + c] * (dp[c] - dl) * sc.ds, sv[32 * h + c + 1] * (dp[c + 1] - dl) * sc.ds,
-                                    whi[c / 2], wlo[c / 2]);
+                    for (int c = 0; c < 32; c += 2) split_half2(dp[32 * h + c], dp[32 * h + c + 1], whi[c / 2], wlo[c / 2]);
                     tmem_st16(ta + 16 * h, whi);
                     tmem_st16(ta + 32 + 16 * h, wlo);
                 }
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&bb.s_empty[g]);
-                    mbar_arrive(&bb.a_full[g]);
-                }
+                if (lane == 0) mbar_arrive(&bb.a_full[g]);
                 ++j;
             }
         }
