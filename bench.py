@@ -316,13 +316,17 @@ def main():
     fwd_flops = qk + 2.0 * D * BLOCK * BLOCK * nnz
     bwd_flops = 10.0 * D * BLOCK * BLOCK * nnz
     if f_ms >= g_ms:
-        dom, dom_flops, dom_ms = "fwd_tc_kernel (entmax_attn_fwd)", fwd_flops, f_ms
+        dom, dom_flops, dom_ms = "fwd_h_kernel (entmax_attn_fwd)", fwd_flops, f_ms
     else:
-        dom, dom_flops, dom_ms = "bwd_dkdv + bwd_dq (entmax_attn_bwd)", bwd_flops, g_ms
+        dom, dom_flops, dom_ms = "bwd_h_dkdv + bwd_h_dq (entmax_attn_bwd)", bwd_flops, g_ms
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    # DRAM bytes (read + write) per call at this workload, from the ncu capture summarised in
+    # profiles/sections_fwd_h_bwd_h_b2h16n16384d64.md (taken at B = 2 and halved)
+    traffic = {"fwd": 183.15e6, "bwd": 440.8e6}["fwd" if f_ms >= g_ms else "bwd"]
     roofline = {"bound": "tensor", "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
-                "frac": achieved / pk_sust, "traffic": None, "kernel": dom,
-                "peak_source": f"{pk_kind} bf16 sustained"}
+                "frac": achieved / pk_sust, "traffic": traffic, "kernel": dom,
+                "peak_source": f"{pk_kind} bf16 sustained",
+                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum, B=2 capture halved"}
 
     # supplementary sweep: contiguous 128-token cluster runs, fewer centres = denser attention
     sweep = []
