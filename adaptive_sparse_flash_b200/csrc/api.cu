@@ -296,6 +296,20 @@ entmax_status bwd_common(const void* Q, const void* K, const void* V, const void
         a.kind = alpha == 1.5f ? kAlpha15 : (alpha == 2.0f ? kAlpha2 : kGeneric);
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (softmax && d == 64) {
+        // dense baseline on the fp16 backward: it makes its own copies of Q, K, V and dO
+        F16Job job;
+        memset(&job, 0, sizeof(job));
+        job.src[0] = Q; job.src[1] = K; job.src[2] = V; job.src[3] = dO;
+        job.dst[0] = ws.Qh; job.dst[1] = ws.Kh; job.dst[2] = ws.Vh; job.dst[3] = ws.dOh;
+        job.maxbits = ws.maxbits;
+        job.n16 = (size_t)B * H * n * d / 8;
+        job.count = 4;
+        a.Qh = ws.Qh; a.Kh = ws.Kh; a.Vh = ws.Vh; a.dOh = ws.dOh; a.maxbits = ws.maxbits;
+        cudaError_t e = launch_to_f16(job, num_sms(), s);
+        if (e == cudaSuccess) e = launch_bwd_h(a, ws.delta_pad, ws.stat_pad, s);
+        return from_cuda(e);
+    }
     if (!softmax && use_f16_path(d, alpha)) {
         // fp16 path: the forward left fp16 copies of Q, K, V and their range exponents in the workspace
         F16Job job;

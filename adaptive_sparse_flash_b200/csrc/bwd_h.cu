@@ -6,6 +6,9 @@
 // block, key block) pairs set in the bit-packed mask are visited ("AdaSplash-2", gist.science (de),
 // section 2, "GPU-Optimierung" and "Bit-Packed Block Mask").
 //
+// The dense softmax baseline uses the same kernels (p = u = softmax probabilities, delta = dO . O, every
+// causal block visited).
+//
 // Both kernels: 352 threads.
 //   warps 0-3, 4-7  compute warpgroups 0 and 1 (thread r of a warpgroup owns row r of the CTA's
 //                   128-row tile, TMEM lane r); block t of the CTA's walk goes to warpgroup t & 1;
@@ -81,10 +84,16 @@ __device__ __forceinline__ bool bar_or256(bool pred) {
     return out != 0;
 }
 
-// p and u of one score: x = cz s - tau (x < 0 off the support).
+// Mode of the dense softmax baseline: p = 2^(x), x = s scale log2(e) - lse log2(e), u = p, delta = dO . O.
+constexpr int kSoftmaxH = 3;
+
+// p and u of one score: x = cz s - tau (x < 0 off the support); softmax: x = c2 s - lse2.
 template <int KIND>
 __device__ __forceinline__ void entmax_pu(float x, float k, float& p, float& u) {
-    if constexpr (KIND == kAlpha15) {
+    if constexpr (KIND == kSoftmaxH) {
+        p = exp2f(x);
+        u = p;
+    } else if constexpr (KIND == kAlpha15) {
         u = fmaxf(x, 0.f);
         p = u * u;
     } else if constexpr (KIND == kAlpha2) {
@@ -202,11 +211,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     volatile int* abort_flag = &bb.abort_flag;
 
     if (tid == 0) init_bars(bb);
-    // query blocks to visit: set in either 64-key half of the tile
+    // query blocks to visit: set in either 64-key half of the tile (entmax), or every block with an
+    // allowed entry (softmax baseline)
     const int J0 = 2 * kt, J1 = 2 * kt + 1;
     for (int w = tid; w < nwq; w += blockDim.x) {
-        uint32_t v = a.maskT[((size_t)bh * a.nkb + J0) * nwq + w];
-        if (J1 < a.nkb) v |= a.maskT[((size_t)bh * a.nkb + J1) * nwq + w];
+        uint32_t v = 0u;
+        if (a.maskT) {
+            v = a.maskT[((size_t)bh * a.nkb + J0) * nwq + w];
+            if (J1 < a.nkb) v |= a.maskT[((size_t)bh * a.nkb + J1) * nwq + w];
+        } else {
+            const int ib = a.causal ? 2 * kt : 0;
+            for (int b = 0; b < 32; ++b) {
+                const int I = w * 32 + b;
+                if (I >= ib && I < a.nqb) v |= 1u << b;
+            }
+        }
         vis[w] = v;
     }
     if (warp == 0) {
@@ -496,8 +515,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) init_bars(bb);
     const int I0 = 2 * qt, I1 = 2 * qt + 1;
     for (int w = tid; w < nw; w += blockDim.x) {
-        uint32_t v = a.mask[((size_t)bh * a.nqb + I0) * nw + w];
-        if (I1 < a.nqb) v |= a.mask[((size_t)bh * a.nqb + I1) * nw + w];
+        uint32_t v = 0u;
+        if (a.mask) {
+            v = a.mask[((size_t)bh * a.nqb + I0) * nw + w];
+            if (I1 < a.nqb) v |= a.mask[((size_t)bh * a.nqb + I1) * nw + w];
+        } else {
+            const int je = a.causal ? min(a.nkb, 2 * qt + 2) : a.nkb;
+            for (int b = 0; b < 32; ++b) {
+                const int J = w * 32 + b;
+                if (J < je) v |= 1u << b;
+            }
+        }
         vis[w] = v;
     }
     if (warp == 0) {
@@ -739,9 +767,10 @@ cudaError_t launch_h_t(const BwdArgs& a, float* delta_pad, float* stat_pad, cuda
 }  // namespace
 
 cudaError_t launch_bwd_h(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaStream_t stream) {
-    if (a.d != 64 || a.softmax || !a.mask || !a.maskT) return cudaErrorInvalidValue;
+    if (a.d != 64 || (!a.softmax && (!a.mask || !a.maskT))) return cudaErrorInvalidValue;
     cudaError_t e = launch_bwd_pre(a, delta_pad, stat_pad, stream);
     if (e != cudaSuccess) return e;
+    if (a.softmax) return launch_h_t<kSoftmaxH>(a, delta_pad, stat_pad, stream);
     if (a.kind == kAlpha15) return launch_h_t<kAlpha15>(a, delta_pad, stat_pad, stream);
     if (a.kind == kAlpha2) return launch_h_t<kAlpha2>(a, delta_pad, stat_pad, stream);
     return launch_h_t<kGeneric>(a, delta_pad, stat_pad, stream);
