@@ -282,12 +282,17 @@ def stats_dict(stats_tensor) -> dict:
     return dict(zip(names, v))
 
 
-def softmax_forward(Q, K, V, causal=True, stream=None):
+def softmax_forward(Q, K, V, causal=True, workspace=None, stream=None):
+    """Dense softmax baseline forward. With a workspace (allocated here when None) d = 64 runs on the
+    fp16 kernels; pass workspace=False for the bf16 kernel."""
     import torch
     B, H, n, d = Q.shape
     O = torch.empty_like(Q)
     lse = torch.empty((B, H, n), dtype=torch.float32, device=Q.device)
-    softmax_attn_fwd(Q, K, V, O, lse, causal, None, stream)
+    if workspace is None:
+        workspace = alloc_workspace(B, H, n, d, _dtype_code(Q), Q.device)
+    opts = make_opts(workspace) if workspace is not False else None
+    softmax_attn_fwd(Q, K, V, O, lse, causal, opts, stream)
     return O, lse
 
 

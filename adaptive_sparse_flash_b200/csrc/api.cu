@@ -356,7 +356,23 @@ EATTN_API entmax_status softmax_attn_fwd(const void* Q, const void* K, const voi
     a.Q = Q; a.K = K; a.V = V; a.O = O; a.lse = lse; a.status = status;
     a.B = B; a.H = H; a.n = n; a.d = d; a.causal = causal; a.ntiles = D.ntiles;
     a.scale = (opts && opts->scale != 0.0f) ? opts->scale : 1.0f / sqrtf((float)d);
-    return from_cuda(launch_softmax_fwd(a, static_cast<cudaStream_t>(stream)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Workspace ws;
+    if (d == 64 && opts && opts->workspace && check_workspace(D, opts, &ws) == ENTMAX_OK) {
+        // fp16 path: copies of Q, K, V in the workspace
+        F16Job job;
+        memset(&job, 0, sizeof(job));
+        job.src[0] = Q; job.src[1] = K; job.src[2] = V;
+        job.dst[0] = ws.Qh; job.dst[1] = ws.Kh; job.dst[2] = ws.Vh;
+        job.maxbits = ws.maxbits;
+        job.n16 = (size_t)B * H * n * d / 8;
+        job.count = 3;
+        a.Qh = ws.Qh; a.Kh = ws.Kh; a.Vh = ws.Vh; a.maxbits = ws.maxbits;
+        cudaError_t e = launch_to_f16(job, num_sms(), s);
+        if (e == cudaSuccess) e = launch_softmax_fwd_h(a, s);
+        return from_cuda(e);
+    }
+    return from_cuda(launch_softmax_fwd(a, s));
 }
 
 EATTN_API entmax_status softmax_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,

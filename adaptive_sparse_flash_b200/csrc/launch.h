@@ -85,7 +85,13 @@ struct SoftmaxFwdArgs {
     int* status;
     int B, H, n, d, causal, ntiles;
     float scale;
+    // fp16 path (softmax_fwd_h.cu, d = 64): copies of Q, K, V and their range exponents
+    const void* Qh;
+    const void* Kh;
+    const void* Vh;
+    const uint32_t* maxbits;
 };
 cudaError_t launch_softmax_fwd(const SoftmaxFwdArgs& a, cudaStream_t stream);
+cudaError_t launch_softmax_fwd_h(const SoftmaxFwdArgs& a, cudaStream_t stream);
 
 }  // namespace eattn

@@ -290,7 +290,7 @@ def main():
     sopts = b.make_opts(ws)
 
     def sm_step():
-        b.softmax_attn_fwd(Q, K, V, O, lse, True, None, stream)
+        b.softmax_attn_fwd(Q, K, V, O, lse, True, sopts, stream)
         b.softmax_attn_bwd(Q, K, V, O, dO, lse, sdQ, sdK, sdV, True, sopts, stream)
 
     def timed(fn, reps):
