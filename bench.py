@@ -322,7 +322,7 @@ def main():
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     # DRAM bytes (read + write) per call at this workload, from the ncu capture summarised in
     # profiles/sections_fwd_h_bwd_h_b2h16n16384d64.md (taken at B = 2 and halved)
-    traffic = {"fwd": 183.15e6, "bwd": 440.8e6}["fwd" if f_ms >= g_ms else "bwd"]
+    traffic = {"fwd": 183.5e6, "bwd": 440.2e6}["fwd" if f_ms >= g_ms else "bwd"]
     roofline = {"bound": "tensor", "achieved": achieved, "peak": pk_sust, "unit": "TFLOP/s",
                 "frac": achieved / pk_sust, "traffic": traffic, "kernel": dom,
                 "peak_source": f"{pk_kind} bf16 sustained",
