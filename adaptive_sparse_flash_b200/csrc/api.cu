@@ -148,8 +148,13 @@ int num_sms() {
     return cache[dev];
 }
 
-// The fp16 forward (fwd_h.cu) serves bf16 inputs with d = 64 and alpha <= 2 (p and u in [0, 1]).
-inline bool use_f16_path(int d, float alpha) { return d == 64 && alpha <= 2.0f; }
+// The fp16 forward (fwd_h.cu) serves bf16 inputs with d = 64 and alpha <= 2 (p and u in [0, 1]), as long as
+// its shared memory (which grows with the number of mask words per row) fits; the backward follows the
+// forward's choice (it reads the forward's fp16 copies).
+constexpr size_t kMaxDynSmem = 232448;
+inline bool use_f16_path(int d, float alpha, int nw) {
+    return d == 64 && alpha <= 2.0f && fwd_h_smem_bytes(nw) <= kMaxDynSmem;
+}
 
 }  // namespace
 }  // namespace eattn
@@ -209,7 +214,7 @@ EATTN_API entmax_status entmax_attn_fwd(const void* Q, const void* K, const void
     cudaError_t e;
     if (dt == ENTMAX_FP32) {
         e = launch_fwd_simt(a, true, s);
-    } else if (use_f16_path(d, alpha)) {
+    } else if (use_f16_path(d, alpha, D.nw)) {
         F16Job job;
         memset(&job, 0, sizeof(job));
         job.src[0] = Q; job.src[1] = K; job.src[2] = V;
@@ -310,7 +315,7 @@ entmax_status bwd_common(const void* Q, const void* K, const void* V, const void
         if (e == cudaSuccess) e = launch_bwd_h(a, ws.delta_pad, ws.stat_pad, s);
         return from_cuda(e);
     }
-    if (!softmax && use_f16_path(d, alpha)) {
+    if (!softmax && use_f16_path(d, alpha, D.nw)) {
         // fp16 path: the forward left fp16 copies of Q, K, V and their range exponents in the workspace
         F16Job job;
         memset(&job, 0, sizeof(job));

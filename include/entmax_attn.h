@@ -90,23 +90,29 @@ size_t entmax_attn_workspace_size(int B, int H, int n, int d, entmax_dtype dt, c
 
 /* Forward. Q, K, V: [B,H,n,d] inputs. O: [B,H,n,d] output (same dtype). tau: float32 [B,H,n]
  * output, the normaliser in z units. block_mask: uint32 output as described above. alpha > 1.
- * causal: 0 or 1. The workspace receives what the backward needs (sum_u, U V, the transposed mask).
- * fp32 uses the FMA path; bf16 uses the tcgen05 path. */
+ * causal: 0 or 1. The workspace receives what the backward needs (sum_u, U V, the transposed mask and,
+ * for bf16 with d = 64 and alpha <= 2, fp16 copies of Q, K, V with their range exponents).
+ * fp32 uses the FMA path. bf16 uses the tcgen05 path: with d = 64 and alpha <= 2 on fp16 operand copies
+ * (exact for bf16 values of magnitude in [2^-14, 2^15), power-of-two scaled beyond), else on bf16
+ * operands with two-term splits. */
 entmax_status entmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* tau,
                               uint32_t* block_mask, int B, int H, int n, int d, float alpha, int causal,
                               entmax_dtype dt, const entmax_opts* opts, void* stream);
 
 /* Backward (bf16 inputs only). Inputs are the forward's inputs and outputs and dO (bf16 [B,H,n,d]); the
- * workspace must be the one the forward filled. Outputs dQ, dK, dV: float32 [B,H,n,d] (fp32 keeps
- * large gradients exact to well below 1e-2; they are accumulated in fp32 TMEM). Visits only the
- * mask's nonzero blocks. */
+ * workspace must be the one the forward filled, after the same Q, K, V (with d = 64 and alpha <= 2 the
+ * backward reads the forward's fp16 copies of them from the workspace). Outputs dQ, dK, dV: float32
+ * [B,H,n,d] (fp32 keeps large gradients exact to well below 1e-2; they are accumulated in fp32 TMEM).
+ * Visits only the mask's nonzero blocks. */
 entmax_status entmax_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                               const float* tau, const uint32_t* block_mask, void* dQ, void* dK, void* dV,
                               int B, int H, int n, int d, float alpha, int causal, entmax_dtype dt,
                               const entmax_opts* opts, void* stream);
 
 /* Dense softmax flash attention in the same library, same tiling: the measurement baseline.
- * lse: float32 [B,H,n] natural-log sum-exp of the scaled scores (output of fwd, input of bwd). */
+ * lse: float32 [B,H,n] natural-log sum-exp of the scaled scores (output of fwd, input of bwd).
+ * With d = 64 and a workspace in opts the forward runs on fp16 operand copies like the entmax forward;
+ * without one (opts NULL) it uses the bf16 kernel. */
 entmax_status softmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* lse,
                                int B, int H, int n, int d, int causal, entmax_dtype dt,
                                const entmax_opts* opts, void* stream);
