@@ -140,6 +140,50 @@ def cpu_baseline(arr):
                       f"{sec:.1f} s, scaled by that head's effective FLOPs", "seconds": sec}
 
 
+def rank_env():
+    """(rank, world size, local rank) from the launcher's environment; one process per GPU."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_ranks(world, backend="nccl", timeout_s=120):
+    """Join the process group when there is more than one rank (a short timeout, so that ranks waiting on
+    one another end with an error)."""
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+
+
+class RankOps:
+    """The only collectives of a run: a barrier around the timed region and the max over ranks of each
+    measured time. The data path has none: every rank computes its own independent heads."""
+
+    def __init__(self, world, device):
+        self.world = world
+        self.device = device
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, x):
+        if self.world == 1:
+            return x
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+
+def whole_job_tflops(world, flops_per_rank, step_ms_max):
+    """Weak scaling: all ranks' effective FLOPs over the slowest rank's time per step."""
+    return world * flops_per_rank / (step_ms_max * 1e-3) / 1e12
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -173,9 +217,7 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     if args.impl == "reference":
         return run_reference(args, rank, world)
 
@@ -188,22 +230,12 @@ def main():
 
     if world > 1:
         torch.cuda.set_device(local)
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    init_ranks(world, "nccl")
     dev = torch.device("cuda", local)
     bld.build()
     b.lib()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ops = RankOps(world, dev)
+    barrier, max_over_ranks = ops.barrier, ops.max
 
     arr = gen_inputs(seed=rank)
     from adaptive_sparse_flash_b200 import inputs as _inputs
@@ -259,7 +291,7 @@ def main():
     bwd_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
     step_ms = sum(f + g for f, g in zip(fwd_ms, bwd_ms)) / args.steps
     step_ms = max_over_ranks(step_ms)
-    value = world * flops / (step_ms * 1e-3) / 1e12
+    value = whole_job_tflops(world, flops, step_ms)
 
     # end to end through the public API with host buffers (pinned), copies inside the timed region
     pin = {k: v.pin_memory() for k, v in host.items()}
@@ -286,7 +318,7 @@ def main():
     torch.cuda.synchronize(dev)
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
-    e2e_val = world * flops / (e2e_ms * 1e-3) / 1e12
+    e2e_val = whole_job_tflops(world, flops, e2e_ms)
 
     # dense softmax baseline on the same inputs, same tiling
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
