@@ -179,6 +179,12 @@ class RankOps:
         return float(t.item())
 
 
+def median(xs):
+    """Middle value of the sorted times (the upper middle for an even count)."""
+    ys = sorted(xs)
+    return ys[len(ys) // 2]
+
+
 def whole_job_tflops(world, flops_per_rank, step_ms_max):
     """Weak scaling: all ranks' effective FLOPs over the slowest rank's time per step."""
     return world * flops_per_rank / (step_ms_max * 1e-3) / 1e12
@@ -330,9 +336,11 @@ def main():
         b.softmax_attn_bwd(Q, K, V, O, dO, lse, sdQ, sdK, sdV, True, sopts, stream)
 
     def timed(fn, reps):
-        fn()
+        """Median of `reps` CUDA-event times after 3 warm-up calls, L2 flushed before each timed call."""
+        for _ in range(3):
+            fn()
         torch.cuda.synchronize(dev)
-        tot = 0.0
+        ts = []
         for _ in range(reps):
             flush.zero_()
             a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -340,10 +348,10 @@ def main():
             fn()
             a1.record(stream)
             torch.cuda.synchronize(dev)
-            tot += a0.elapsed_time(a1)
-        return tot / reps
+            ts.append(a0.elapsed_time(a1))
+        return median(ts)
 
-    softmax_ms = max_over_ranks(timed(sm_step, 3))
+    softmax_ms = max_over_ranks(timed(sm_step, 7))
 
     # roofline of the dominant kernel call (tensor-bound): algorithmic FLOPs per launch / its time
     pk_burst, pk_sust, hbm, pk_kind = peaks()
@@ -374,8 +382,8 @@ def main():
             step()
             torch.cuda.synchronize(dev)
             nz = int(np.unpackbits(mask.cpu().numpy().view(np.uint8), bitorder="little").sum())
-            ms_e = timed(step, 3)
-            ms_s = timed(sm_step, 3)
+            ms_e = timed(step, 7)
+            ms_s = timed(sm_step, 7)
             fl = effective_flops(N, D, B * H, nz)
             sweep.append({"centres": c, "block_sparsity": 1.0 - nz / causal_blocks, "entmax_ms": ms_e,
                           "softmax_ms": ms_s, "eff_tflops": fl / (ms_e * 1e-3) / 1e12,

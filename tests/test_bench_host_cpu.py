@@ -124,3 +124,9 @@ def test_effective_flops():
     assert bench.effective_flops(128, d, 1, 0, causal=False) == 2.0 * d * 128 * 128
     # each nonzero block adds P V (2 d per entry) and the five backward products (10 d per entry)
     assert bench.effective_flops(128, d, 1, 7) - bench.effective_flops(128, d, 1, 0) == 12.0 * d * blk * blk * 7
+
+
+def test_median_of_repetitions():
+    # one slow repetition (another tenant, a clock dip) does not move the reported time
+    assert bench.median([2.5, 2.4, 9.0, 2.6, 2.5, 2.45, 2.55]) == 2.5
+    assert bench.median([3.0]) == 3.0
