@@ -125,7 +125,7 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 }
 
 // ---------------------------------------------------------------------------------------------
-// TMA (tiled, no multicast: every CTA loads its own tiles from this GPU's memory)
+// TMA (tiled; every CTA loads its own tiles from this GPU's memory)
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
