@@ -409,7 +409,7 @@ def main():
                        "pct_bf16_peak": value / world / pk_sust * 100.0},
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps * world,  # every rank launches its own
             "clocks": clk.summary(),
             "roofline": roofline,
             "cpu_baseline": cpu,
