@@ -57,6 +57,7 @@ class EntmaxStats(ctypes.Structure):
         ("nonzero_blocks", ctypes.c_ulonglong),
         ("sweeps", ctypes.c_ulonglong),
         ("overflow_rows", ctypes.c_ulonglong),
+        ("support", ctypes.c_ulonglong),
     ]
 
 
@@ -74,6 +75,8 @@ class EntmaxOpts(ctypes.Structure):
         ("stats", ctypes.c_void_p),
         ("tau_hist", ctypes.c_void_p),
         ("steps", ctypes.c_void_p),
+        ("events", ctypes.c_void_p),
+        ("num_events", ctypes.c_int),
     ]
 
 
@@ -147,7 +150,9 @@ def _dtype_code(t) -> int:
 
 
 def make_opts(workspace=None, *, scale=0.0, mask_block=0, hist_bins=0, init_mode=0,
-              stats=None, tau_hist=None, steps=None) -> EntmaxOpts:
+              stats=None, tau_hist=None, steps=None, events=None) -> EntmaxOpts:
+    """Options block. `events`: torch.cuda.Event objects (already recorded once, so that their CUDA handles
+    exist) that the call records around its kernel launches (include/entmax_attn.h, per-kernel timing)."""
     o = EntmaxOpts()
     o.scale = float(scale)
     o.mask_block = int(mask_block)
@@ -159,6 +164,11 @@ def make_opts(workspace=None, *, scale=0.0, mask_block=0, hist_bins=0, init_mode
     o.stats = None if stats is None else stats.data_ptr()
     o.tau_hist = None if tau_hist is None else tau_hist.data_ptr()
     o.steps = None if steps is None else steps.data_ptr()
+    if events:
+        arr = (ctypes.c_void_p * len(events))(*[int(e.cuda_event) for e in events])
+        o.events = ctypes.cast(arr, ctypes.c_void_p)
+        o.num_events = len(events)
+        o._keep = arr  # the handle array must outlive the call
     return o
 
 
@@ -278,7 +288,7 @@ def backward(Q, K, V, fwd: EntmaxForward, dO, stream=None):
 def stats_dict(stats_tensor) -> dict:
     v = [int(x) for x in stats_tensor.cpu().tolist()]
     names = ["rows", "steps", "fallbacks"] + [f"step_hist_{i}" for i in range(9)] + \
-        ["causal_blocks", "candidate_blocks", "nonzero_blocks", "sweeps", "overflow_rows"]
+        ["causal_blocks", "candidate_blocks", "nonzero_blocks", "sweeps", "overflow_rows", "support"]
     return dict(zip(names, v))
 
 

@@ -17,6 +17,40 @@ namespace eattn {
 
 __device__ int g_status;  // ENTMAX_OK, or the first device-side error since the last check
 
+// Timing events of the API call running on this host thread (entmax_opts.events): event i is recorded right
+// before the call's i-th kernel launch, and one more after its last launch.
+namespace {
+struct EventTrail {
+    void* const* events = nullptr;
+    int count = 0;
+    int next = 0;
+};
+thread_local EventTrail t_trail;
+
+// Installs the trail of one API call for its duration; the destructor records the closing event.
+struct TrailScope {
+    cudaStream_t stream;
+    TrailScope(const entmax_opts* o, cudaStream_t s) : stream(s) {
+        t_trail = EventTrail{};
+        if (o && o->events && o->num_events > 0) {
+            t_trail.events = o->events;
+            t_trail.count = o->num_events;
+        }
+    }
+    ~TrailScope() {
+        launch_mark(stream);
+        t_trail = EventTrail{};
+    }
+};
+}  // namespace
+
+void launch_mark(cudaStream_t stream) {
+    if (t_trail.events && t_trail.next < t_trail.count) {
+        cudaEvent_t ev = static_cast<cudaEvent_t>(t_trail.events[t_trail.next++]);
+        if (ev) cudaEventRecord(ev, stream);
+    }
+}
+
 namespace {
 
 // A kernel that waits on a barrier nobody arrives at, bounded by limit_ns: exercises the timeout path.
@@ -69,9 +103,10 @@ entmax_status check_dims(int B, int H, int n, int d, entmax_dtype dt, const entm
     if (mb != 32 && mb != 64) return ENTMAX_ERR_UNSUPPORTED;
     if (dt == ENTMAX_BF16 && mb != 64) return ENTMAX_ERR_UNSUPPORTED;
     const int bins = (o && o->hist_bins) ? o->hist_bins : 256;
-    if (bins != 64 && bins != 128 && bins != 256) return ENTMAX_ERR_UNSUPPORTED;
+    if (bins != 64 && bins != 128 && bins != 256 && bins != 512) return ENTMAX_ERR_UNSUPPORTED;
     if (o && (o->init_mode < 0 || o->init_mode > 1)) return ENTMAX_ERR_INVALID;
     if (o && o->scale != 0.0f && !(o->scale > 0.0f && isfinite(o->scale))) return ENTMAX_ERR_INVALID;
+    if (o && (o->num_events < 0 || (o->num_events > 0 && !o->events))) return ENTMAX_ERR_INVALID;
     Dims D;
     D.B = B; D.H = H; D.n = n; D.d = d; D.mb = mb; D.bins = bins;
     D.nqb = (n + mb - 1) / mb;
@@ -149,11 +184,11 @@ int num_sms() {
 }
 
 // The fp16 forward (fwd_h.cu) serves bf16 inputs with d = 64 and alpha <= 2 (p and u in [0, 1]), as long as
-// its shared memory (which grows with the number of mask words per row) fits; the backward follows the
-// forward's choice (it reads the forward's fp16 copies).
+// its shared memory (which grows with the number of mask words per row and with the histogram size) fits;
+// the backward follows the forward's choice (it reads the forward's fp16 copies).
 constexpr size_t kMaxDynSmem = 232448;
-inline bool use_f16_path(int d, float alpha, int nw) {
-    return d == 64 && alpha <= 2.0f && fwd_h_smem_bytes(nw) <= kMaxDynSmem;
+inline bool use_f16_path(int d, float alpha, int nw, int bins) {
+    return d == 64 && alpha <= 2.0f && fwd_h_smem_bytes(nw, bins) <= kMaxDynSmem;
 }
 
 }  // namespace
@@ -165,7 +200,7 @@ using namespace eattn;
 
 extern "C" {
 
-EATTN_API int entmax_attn_version(void) { return 1; }
+EATTN_API int entmax_attn_version(void) { return 2; }
 
 EATTN_API const char* entmax_status_str(entmax_status s) {
     switch (s) {
@@ -210,11 +245,13 @@ EATTN_API entmax_status entmax_attn_fwd(const void* Q, const void* K, const void
     const float scale = opts->scale != 0.0f ? opts->scale : 1.0f / sqrtf((float)d);
     a.sp = make_solve_params(alpha, scale, D.bins, opts->init_mode);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-
+    // 512 bins fit only the fp16 forward's shared-memory plan
+    if (D.bins > 256 && !(dt == ENTMAX_BF16 && use_f16_path(d, alpha, D.nw, D.bins))) return ENTMAX_ERR_UNSUPPORTED;
+    TrailScope trail(opts, s);
     cudaError_t e;
     if (dt == ENTMAX_FP32) {
         e = launch_fwd_simt(a, true, s);
-    } else if (use_f16_path(d, alpha, D.nw)) {
+    } else if (use_f16_path(d, alpha, D.nw, D.bins)) {
         F16Job job;
         memset(&job, 0, sizeof(job));
         job.src[0] = Q; job.src[1] = K; job.src[2] = V;
@@ -301,6 +338,7 @@ entmax_status bwd_common(const void* Q, const void* K, const void* V, const void
         a.kind = alpha == 1.5f ? kAlpha15 : (alpha == 2.0f ? kAlpha2 : kGeneric);
     }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TrailScope trail(opts, s);
     if (softmax && d == 64) {
         // dense baseline on the fp16 backward: it makes its own copies of Q, K, V and dO
         F16Job job;
@@ -315,7 +353,7 @@ entmax_status bwd_common(const void* Q, const void* K, const void* V, const void
         if (e == cudaSuccess) e = launch_bwd_h(a, ws.delta_pad, ws.stat_pad, s);
         return from_cuda(e);
     }
-    if (!softmax && use_f16_path(d, alpha, D.nw)) {
+    if (!softmax && use_f16_path(d, alpha, D.nw, D.bins)) {
         // fp16 path: the forward left fp16 copies of Q, K, V and their range exponents in the workspace
         F16Job job;
         memset(&job, 0, sizeof(job));
@@ -362,6 +400,7 @@ EATTN_API entmax_status softmax_attn_fwd(const void* Q, const void* K, const voi
     a.B = B; a.H = H; a.n = n; a.d = d; a.causal = causal; a.ntiles = D.ntiles;
     a.scale = (opts && opts->scale != 0.0f) ? opts->scale : 1.0f / sqrtf((float)d);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    TrailScope trail(opts, s);
     Workspace ws;
     if (d == 64 && opts && opts->workspace && check_workspace(D, opts, &ws) == ENTMAX_OK) {
         // fp16 path: copies of Q, K, V in the workspace

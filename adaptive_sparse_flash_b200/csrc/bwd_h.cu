@@ -1,10 +1,18 @@
 // bwd_h.cu - backward of alpha-entmax attention for alpha <= 2 and d = 64 on the sm_100a tensor cores,
 // from fp16 copies of Q, K, V (made by the forward) and dO (f16.cu).
 //
-// With g = dO V^T, u = [z - tau]_+^(k-1) and delta = (dO . U V) / sum(u) (bwd_tc.cu: bwd_pre), the score
-// gradient is dS = u (g - delta); dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO. Only the (query
-// block, key block) pairs set in the bit-packed mask are visited ("AdaSplash-2", gist.science (de),
-// section 2, "GPU-Optimierung" and "Bit-Packed Block Mask").
+// With g = dO V^T, u = [z - tau]_+^(k-1) and delta = sum(u g) / sum(u), the score gradient is
+// dS = u (g - delta); dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO. Only the (query block, key block)
+// pairs set in the bit-packed mask are visited ("AdaSplash-2", gist.science (de), section 2,
+// "GPU-Optimierung" and "Bit-Packed Block Mask").
+//
+// delta: bwd_pre (bwd_tc.cu) forms an estimate d~ = dO . (U V) / sum u from the forward's U V, whose U was
+// one fp16 term. bwd_h_dq runs first and uses that estimate for its dS~ = u (g - d~); while it walks a query
+// row's nonzero blocks it also sums dS~ over the row in fp32, which gives the exact delta:
+// sum_j u_j (g_j - d~) = sum u (delta - d~), so delta = d~ + sum_j dS~_j / sum u (sum u from the forward,
+// over the same u: both passes form x = fma(s, cz, -tau) from the same score tile). It writes that delta
+// back for bwd_h_dkdv, which runs second, since dK sums dS against query rows that can be large; in dQ the
+// estimate's small error is damped by the unit-scale keys.
 //
 // The dense softmax baseline uses the same kernels (p = u = softmax probabilities, delta = dO . O, every
 // causal block visited).
@@ -498,11 +506,12 @@ template <int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_h_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                    const BwdArgs a, const float* __restrict__ delta_pad, const float* __restrict__ stat_pad) {
+                    const BwdArgs a, float* __restrict__ delta_pad, const float* __restrict__ stat_pad) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = align_smem_1024(smem_raw);
     Bars& bb = *reinterpret_cast<Bars*>(smem + qOffBar);
-    uint32_t* vis = reinterpret_cast<uint32_t*>(&bb + 1);  // [nw] key blocks to visit
+    float* xsum = reinterpret_cast<float*>(&bb + 1);          // [TM]: warpgroup 1's row sums of dS~
+    uint32_t* vis = reinterpret_cast<uint32_t*>(xsum + TM);     // [nw] key blocks to visit
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qt = (int)gridDim.x - 1 - (int)blockIdx.x;
@@ -630,6 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Scales sc = make_scales(a);
         const float tau = stat_pad[(size_t)bh * npad + min(row, npad - 1)];
         const float dl = delta_pad[(size_t)bh * npad + min(row, npad - 1)] * sc.dl;
+        float rs = 0.f;  // this warpgroup's share of the row sum of u (g - d~), in dP units
         bool ok = true;
         int t = 0;
         uint32_t j = 0;
@@ -679,7 +689,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bb.d_empty[g]);
 #pragma unroll
-                for (int c = 0; c < TB; ++c) dp[c] = sv[c] * (dp[c] - dl) * sc.ds;
+                for (int c = 0; c < TB; ++c) {
+                    const float e = sv[c] * (dp[c] - dl);
+                    if constexpr (KIND != kSoftmaxH) rs += e;
+                    dp[c] = e * sc.ds;
+                }
                 ok = __all_sync(0xffffffffu, wait_bounded(&bb.a_empty[g], (j & 1) ^ 1, abort_flag, a.status));
                 if (!ok) break;
                 const uint32_t ta = lane_base + 256u + 64u * g;
@@ -698,7 +712,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++j;
             }
         }
+        if (g == 1) xsum[r] = rs;
         ok = !bar_or256(!ok || *abort_flag != 0);
+        if constexpr (KIND != kSoftmaxH) {
+            // the exact delta of this row, for the dK / dV kernel that runs next
+            if (ok && g == 0 && qvalid) {
+                const float s_u = a.sum_u[(size_t)bh * a.n + row];
+                const float corr = s_u > 0.f ? (rs + xsum[r]) / s_u : 0.f;
+                delta_pad[(size_t)bh * npad + row] = (dl + corr) / sc.dl;
+            }
+        }
         if (T > 0 && ok) ok = __all_sync(0xffffffffu, wait_bounded(&bb.acc_full, 0, abort_flag, a.status));
         ok = !bar_or256(!ok || *abort_flag != 0);
         // warpgroup g writes columns 32 g .. 32 g + 31 of dQ
@@ -743,22 +766,25 @@ cudaError_t launch_h_t(const BwdArgs& a, float* delta_pad, float* stat_pad, cuda
     if ((e = make_tmap_f16(&tk64, a.Kh, BH, a.n, D, TB)) != cudaSuccess) return e;
     if ((e = make_tmap_f16(&tv64, a.Vh, BH, a.n, D, TB)) != cudaSuccess) return e;
     const int ntiles = (a.n + TM - 1) / TM;
+    // dQ first: it writes the exact delta of every row (entmax), which the dK / dV kernel then reads
+    {
+        const size_t bytes = 1024 + qOffBar + sizeof(Bars) + TM * sizeof(float) + (size_t)a.nw * 4;
+        if (bytes > 232448) return cudaErrorInvalidConfiguration;
+        auto kern = bwd_h_dq_kernel<KIND>;
+        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
+            return e;
+        launch_mark(stream);
+        kern<<<dim3(ntiles, BH), kThreads, bytes, stream>>>(tq128, tk64, tv64, tdo128, a, delta_pad, stat_pad);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     {
         const size_t bytes = 1024 + kvOffBar + sizeof(Bars) + (size_t)a.nwq * 4;
         if (bytes > 232448) return cudaErrorInvalidConfiguration;
         auto kern = bwd_h_dkdv_kernel<KIND>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
             return e;
+        launch_mark(stream);
         kern<<<dim3(ntiles, BH), kThreads, bytes, stream>>>(tq64, tk128, tv128, tdo64, a, delta_pad, stat_pad);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    {
-        const size_t bytes = 1024 + qOffBar + sizeof(Bars) + (size_t)a.nw * 4;
-        if (bytes > 232448) return cudaErrorInvalidConfiguration;
-        auto kern = bwd_h_dq_kernel<KIND>;
-        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
-            return e;
-        kern<<<dim3(ntiles, BH), kThreads, bytes, stream>>>(tq128, tk64, tv64, tdo128, a, delta_pad, stat_pad);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;

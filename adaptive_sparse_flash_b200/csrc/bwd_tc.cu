@@ -736,6 +736,7 @@ cudaError_t launch_t(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaSt
     {
         const int warps = 8;
         dim3 grid((a.nqb * TB + warps - 1) / warps, BH);
+        launch_mark(stream);
         bwd_pre_kernel<D><<<grid, warps * 32, 0, stream>>>(a, delta_pad, stat_pad);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -755,6 +756,7 @@ cudaError_t launch_t(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaSt
         auto kern = bwd_dkdv_kernel<D, MODE, SPLIT>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
             return e;
+        launch_mark(stream);
         kern<<<dim3(ntiles, BH), kThreads, bytes, stream>>>(tq64, tk128, tv128, tdo64, a, delta_pad, stat_pad);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -764,6 +766,7 @@ cudaError_t launch_t(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaSt
         auto kern = bwd_dq_kernel<D, MODE, SPLIT>;
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
             return e;
+        launch_mark(stream);
         kern<<<dim3(ntiles, BH), kThreads, bytes, stream>>>(tq128, tk64, tv64, tdo128, a, delta_pad, stat_pad);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
@@ -783,6 +786,7 @@ cudaError_t launch_d(const BwdArgs& a, float* dp, float* sp, cudaStream_t s) {
 cudaError_t launch_bwd_pre(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaStream_t stream) {
     const int warps = 8;
     dim3 grid((a.nqb * TB + warps - 1) / warps, a.B * a.H);
+    launch_mark(stream);
     if (a.d == 64) bwd_pre_kernel<64><<<grid, warps * 32, 0, stream>>>(a, delta_pad, stat_pad);
     else bwd_pre_kernel<128><<<grid, warps * 32, 0, stream>>>(a, delta_pad, stat_pad);
     return cudaGetLastError();

@@ -83,28 +83,30 @@ __device__ __forceinline__ void add_sums(float x, float k, float& F0, float& F1,
 // Histogram ring (thread-owned row).
 //   hist  u16 [B slots][128 rows]; counts saturate at 65535 (a saturated count only drops entries,
 //         which keeps the bound);
-//   live  u32 [128 rows][kLiveStride]: bit s of row r's 8 words marks slot s as holding a counted bin
-//         of the current window. Sliding the window clears bits instead of counts, so the histogram
-//         needs no zeroing and a slide costs a few word operations.
+//   live  u32 [128 rows][stride]: bit s of row r's B / 32 words (8 for B <= 256, 16 for B = 512) marks
+//         slot s as holding a counted bin of the current window. Sliding the window clears bits instead
+//         of counts, so the histogram needs no zeroing and a slide costs a few word operations.
 // ---------------------------------------------------------------------------------------------
-constexpr int kLiveStride = 9;  // words per row (8 used; odd stride keeps rows on distinct banks)
+constexpr int kLiveStride = 9;      // words per row for B <= 256 (8 used; odd stride: rows on distinct banks)
+constexpr int kLiveStride512 = 17;  // words per row for B = 512 (16 used)
 
 struct HistRow {
     float m_raw;     // running max of the raw score
     float thr_raw;   // raw threshold for binning: z > m_run - 1
     int top;         // bin index of the running max
     bool any;        // any entry seen
+    int nlw;         // live words per row (stride - 1)
     uint32_t* live;  // this row's live words in shared memory
 };
 
-__device__ __forceinline__ void hist_init(HistRow& h, uint32_t* live_all, int r) {
+__host__ __device__ __forceinline__ void hist_init(HistRow& h, uint32_t* live_all, int r, int stride = kLiveStride) {
     h.m_raw = -INFINITY;
     h.thr_raw = INFINITY;
     h.top = 0;
     h.any = false;
-    h.live = live_all + r * kLiveStride;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) h.live[i] = 0u;
+    h.nlw = stride - 1;
+    h.live = live_all + r * stride;
+    for (int i = 0; i < h.nlw; ++i) h.live[i] = 0u;
 }
 
 __device__ __forceinline__ int bin_of(float a, float cbin) {
@@ -112,7 +114,8 @@ __device__ __forceinline__ int bin_of(float a, float cbin) {
     return __float2int_rd(y);
 }
 
-// Bits [s0, s0 + len) of a B-bit ring (B <= 256, a power of two, len < B) as 8 words (host-testable).
+// Word i of the bits [s0, s0 + len) of a B-bit ring (B a power of two, 32 <= B <= 512, len < B; words at
+// or beyond B / 32 are 0), host-testable.
 __host__ __device__ __forceinline__ uint32_t ring_word_mask(int i, int s0, int len, int B) {
     const int lo = i * 32;
     if (lo >= B) return 0u;
@@ -134,12 +137,10 @@ __device__ __forceinline__ void hist_raise(HistRow& h, float a_max, float cbin, 
     if (h.any && nt > h.top) {
         const int d = nt - h.top;
         if (d >= B) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) h.live[i] = 0u;
+            for (int i = 0; i < h.nlw; ++i) h.live[i] = 0u;
         } else {
             const int s0 = (h.top + 1) & (B - 1);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
+            for (int i = 0; i < h.nlw; ++i) {
                 const uint32_t m = ring_word_mask(i, s0, d, B);
                 if (m) h.live[i] &= ~m;
             }
@@ -203,8 +204,7 @@ __device__ __forceinline__ void stash_add(Stash& st, float a, float thr_raw, flo
 // the row switches to streaming the histogram.
 __device__ __forceinline__ void hist_from_stash(HistRow& h, const Stash& st, const float* stash, float m_raw,
                                                 float thr_raw, float cbin, int B, uint16_t* hist, int r) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) h.live[i] = 0u;
+    for (int i = 0; i < h.nlw; ++i) h.live[i] = 0u;
     h.any = m_raw > -INFINITY;
     h.m_raw = m_raw;
     h.thr_raw = thr_raw;
@@ -268,9 +268,6 @@ __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, cons
             while (Ak(t) < thr) ++t;
             return t;
         };
-        uint32_t lw[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) lw[i] = h.live[i];
         const int stop = h.top & (B - 1);
         const int nw = B >= 32 ? B / 32 : 1;
         int J = B - 1, J0 = 0;  // moments are evaluated at J0 (bins with offset < J0)
@@ -278,9 +275,7 @@ __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, cons
         // visit slots stop, stop-1, ..., 0, B-1, ..., stop+1: word by word from the word holding `stop`
         for (int step = 0; step <= nw && !found; ++step) {
             const int wi = ((stop >> 5) - step + 2 * nw) % nw;
-            uint32_t bits = 0u;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) bits = (i == wi) ? lw[i] : bits;
+            uint32_t bits = h.live[wi];
             if (B < 32) bits &= (1u << B) - 1u;
             if (step == 0) bits &= (stop & 31) == 31 ? 0xffffffffu : ((2u << (stop & 31)) - 1u);   // slots <= stop
             if (step == nw) bits &= (stop & 31) == 31 ? 0u : ~((2u << (stop & 31)) - 1u);        // slots > stop

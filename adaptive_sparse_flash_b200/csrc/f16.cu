@@ -81,8 +81,10 @@ cudaError_t launch_to_f16(const F16Job& job, int num_sms, cudaStream_t stream) {
     // memory-bound copy: 8 resident blocks of 256 threads per SM, grid-stride
     const size_t want = (job.n16 + kCvtThreads - 1) / kCvtThreads;
     const int grid1 = (int)(want < (size_t)num_sms * 8 ? (want > 0 ? want : 1) : (size_t)num_sms * 8);
+    launch_mark(stream);
     to_f16_pass1<<<grid1, kCvtThreads, 0, stream>>>(job);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    launch_mark(stream);
     to_f16_pass2<<<num_sms, kCvtThreads, 0, stream>>>(job);
     return cudaGetLastError();
 }

@@ -41,9 +41,18 @@ __device__ __forceinline__ int allowed_keys(int row, int n, int causal) {
     return causal ? min(row + 1, n) : n;
 }
 
+// Mask blocks (query block, key block) with at least one allowed entry, over query blocks qb0 .. qb0 + nq - 1
+// of a tile (causal: key blocks 0 .. qb, since query and key blocks have the same size).
+__device__ __forceinline__ uint32_t tile_causal_blocks(int qb0, int nq, int nqb, int nkb, int causal) {
+    uint32_t c = 0;
+    for (int qb = qb0; qb < qb0 + nq && qb < nqb; ++qb) c += (uint32_t)(causal ? min(qb + 1, nkb) : nkb);
+    return c;
+}
+
 // Per-CTA statistics, reduced into entmax_stats at the end of a tile.
 struct TileStats {
     uint32_t rows, steps, fallbacks, candidate_blocks, nonzero_blocks, causal_blocks, sweeps, overflow_rows;
+    uint32_t support;  // nonzero probabilities of the tile's rows
     uint32_t step_hist[kMaxSteps + 1];
 };
 
@@ -57,6 +66,7 @@ __device__ __forceinline__ void flush_stats(entmax_stats* g, const TileStats& t)
     atomicAdd(&g->causal_blocks, (unsigned long long)t.causal_blocks);
     atomicAdd(&g->sweeps, (unsigned long long)t.sweeps);
     if (t.overflow_rows) atomicAdd(&g->overflow_rows, (unsigned long long)t.overflow_rows);
+    atomicAdd(&g->support, (unsigned long long)t.support);
     for (int i = 0; i <= kMaxSteps; ++i)
         if (t.step_hist[i]) atomicAdd(&g->step_hist[i], (unsigned long long)t.step_hist[i]);
 }

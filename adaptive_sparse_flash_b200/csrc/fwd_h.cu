@@ -4,23 +4,24 @@
 // One CTA per (b, h, 128-row query tile), 352 threads:
 //   warps 0-3, 4-7  compute warpgroups 0 and 1. Thread r of a warpgroup owns query row r of the tile
 //                   and reads TMEM lane r; the two warpgroups take alternate key blocks of every sweep;
-//   warp 8          S issue (one thread): S = Q K^T from shared memory into two TMEM buffers per
+//   warp 8          S issue (one thread): S = Q K^T from shared memory into three TMEM buffers per
 //                   warpgroup;
 //   warp 10         P V issue (one thread): O += P V and Obar += U V with P and U stored by the compute
 //                   warps into the TMEM columns of the S tile they came from. Two issuing threads keep the
 //                   tensor pipe fed: each waits only on its own barriers, in block order;
 //   warp 9          TMA issue (one thread): Q once, K blocks of 64 keys and, in P V sweeps, V blocks.
 //
-// P and U lie in [0, 1] for alpha <= 2. P enters P V as one fp16 term (11 significant bits; bf16 would
-// need a two-term split). U enters as two fp16 terms, U = hi + lo: U V only feeds the backward's
-// delta = dO . (U V) / sum u, which shifts every dS of its row, so it is kept to ~22 bits. P and U hi
-// of a 64-key block fit the 64 columns of its S tile; U lo goes to a 32-column buffer paired with it. A new S tile goes into a buffer only after the P V products that read its
-// previous P and U have completed (a commit barrier per buffer), and the MMA thread waits for all P V
-// products at the end of a P V sweep: MMAs into different accumulators are not ordered by issue alone.
+// P and U lie in [0, 1] for alpha <= 2 and each enters its product as one fp16 term (11 significant bits;
+// bf16 would need a two-term split). U V only gives the backward a first estimate of
+// delta = dO . (U V) / sum u for its dQ kernel, which then accumulates the exact delta from fp32 u and g
+// (bwd_h.cu); so one term is enough here. P and U of a 64-key block fit the 64 columns of its S tile. A
+// new S tile goes into a buffer only after the P V products that read its previous P and U have
+// completed (a commit barrier per buffer), and the MMA thread waits for all P V products at the end of a
+// P V sweep: MMAs into different accumulators are not ordered by issue alone.
 //
-// TMEM columns (512): S buffer b of warpgroup g at 64 (2 g + b), holding P (first 32 columns) and U hi
-// (next 32; K step kk of 16 keys is columns 8 kk .. 8 kk + 7 of each) in P V sweeps; the U lo of that
-// buffer at 256 + 32 (2 g + b); O at 384, Obar at 448.
+// TMEM columns (512): S buffer b (of three) of warpgroup g at 64 (3 g + b), holding P (first 32 columns)
+// and U (next 32; K step kk of 16 keys is columns 8 kk .. 8 kk + 7 of each) in P V sweeps; O at 384, U V at
+// 448.
 //
 // Sweeps follow the plan protocol of the bf16 forward (fwd_tc.cu): before each sweep the compute warps
 // publish its kind and its set of key blocks, which the issuing warps follow.
@@ -55,25 +56,33 @@ constexpr int kThreads = 352;
 constexpr int kCompute = 256;
 constexpr int NKS = 4;
 constexpr int NVS = 8;
-constexpr int kHalf = 88;  // stash entries per row and warpgroup
+constexpr int NSB = 3;  // S buffers per compute warpgroup
 
 constexpr uint64_t kDescK = sdesc_sw128_fields(16, 1024);
 constexpr uint64_t kDescMN = sdesc_sw128_fields(64 * 128, 1024);
 
 constexpr uint32_t kKBytes = BN * D * 2;                 // 8 KB per K or V block
-constexpr uint32_t kHistBytes = 256u * BM * 2u;          // u16 [256][128]
-constexpr uint32_t kStashBytes = 2u * kHalf * BM * 4u;   // fp32 [2][kHalf][128]
 constexpr uint32_t kQBytes = BM * D * 2;                 // 16 KB
 constexpr uint32_t offQ = 0;
 constexpr uint32_t offK = offQ + kQBytes;
 constexpr uint32_t offHist = offK + NKS * kKBytes;
-constexpr uint32_t offStash = offHist + kHistBytes;
-constexpr uint32_t offV = offHist;  // the V ring reuses the histogram (dead in P V sweeps)
-constexpr uint32_t offSmall = offStash + kStashBytes;
-static_assert(NVS * kKBytes <= kHistBytes, "V ring must fit the histogram region");
+
+// Shared-memory plan for up to NB histogram bins (256, or 512): the histogram u16 [NB][128] (the V ring of
+// P V sweeps reuses it), then the candidate stash fp32 [2][kHalf][128]. At 512 bins the histogram takes
+// 128 KB and the stash shrinks to 28 entries per row and warpgroup, so that the CTA still fits.
+template <int NB>
+struct HCfg {
+    static constexpr int kHalf = NB == 512 ? 28 : 88;  // stash entries per row and warpgroup
+    static constexpr uint32_t kHistBytes = (uint32_t)NB * BM * 2u;
+    static constexpr uint32_t kStashBytes = 2u * kHalf * BM * 4u;
+    static constexpr uint32_t offStash = offHist + kHistBytes;
+    static constexpr uint32_t offV = offHist;
+    static constexpr uint32_t offSmall = offStash + kStashBytes;
+    static constexpr int kStride = NB == 512 ? kLiveStride512 : kLiveStride;  // live words per row + 1
+    static_assert(NVS * kKBytes <= kHistBytes, "V ring must fit the histogram region");
+};
 
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColUlo = 256;
 constexpr uint32_t kColO = 384;
 constexpr uint32_t kColOb = 448;
 
@@ -84,16 +93,17 @@ enum : int {
     kXTau = 3, kXTau2 = 4, kXLo = 5, kXTwo = 6,  // solver state broadcast by warpgroup 0
     kXF0 = 7, kXF1 = 8, kXF2 = 9, kXF0b = 10,    // partial sums of warpgroup 1
     kXOvf = 11,                                  // 1: the row's candidates did not fit the stash
-    kXRows = 12
+    kXCnt = 12,                                  // partial support count of warpgroup 1 (int bits)
+    kXRows = 13
 };
 
 struct Small {
     uint64_t q_full;
     uint64_t k_full[NKS], k_empty[NKS];
     uint64_t v_full[NVS], v_empty[NVS];
-    uint64_t s_full[2][2], s_empty[2][2];  // [warpgroup][buffer]
-    uint64_t pv_free[2][2];                // P V products that read a buffer's P and U have completed
-    uint64_t pu_full[2][2];                // a buffer's P and U are stored (one barrier per buffer, so
+    uint64_t s_full[2][NSB], s_empty[2][NSB];  // [warpgroup][buffer]
+    uint64_t pv_free[2][NSB];                  // P V products that read a buffer's P and U have completed
+    uint64_t pu_full[2][NSB];                  // a buffer's P and U are stored (one barrier per buffer, so
                                            // that no barrier runs two phases ahead of its waiter)
     uint64_t o_full;
     uint64_t ctrl;
@@ -102,9 +112,9 @@ struct Small {
     int abort_flag;
     int plan_kind[2];
     TileStats st;
-    float T[260];
+    float T[516];  // i^k for i = 0 .. bins (generic alpha)
     float xf[kXRows][BM];
-    // followed by: plan_bits[2][W], next[W], mrow[2][W], live[128][kLiveStride]
+    // followed by: plan_bits[2][W], next[W], mrow[2][W], live[128][stride]
 };
 
 // OR of `pred` over the 256 compute threads (named barrier 1); every compute thread gets the result.
@@ -129,19 +139,18 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 // Drop the entries of a stash half at or below thr. Returns the new count, or -1 (overflow) when more
 // than half of the half stays occupied, so that pruning stays amortised O(1) per entry.
-static __device__ __noinline__ int stash_prune(int n, float* st, int r, float thr) {
+static __device__ __noinline__ int stash_prune(int n, float* st, int r, float thr, int half) {
     int j = 0;
     for (int i = 0; i < n; ++i) {
         const float v = st[i * BM + r];
         if (v > thr) st[(j++) * BM + r] = v;
     }
-    return j > kHalf / 2 ? -1 : j;
+    return j > half / 2 ? -1 : j;
 }
 
 // Start row r's histogram with its window top at the bin of the final max m_raw.
 __device__ __forceinline__ void hist_start(HistRow& h, float m_raw, const SolveParams& sp) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) h.live[i] = 0u;
+    for (int i = 0; i < h.nlw; ++i) h.live[i] = 0u;
     h.any = m_raw > -INFINITY;
     h.m_raw = m_raw;
     h.thr_raw = m_raw - sp.inv_cz;
@@ -176,14 +185,21 @@ template <int KIND>
 __device__ __forceinline__ void half_sums(const float* st, int n, int r, const SolveParams& sp, float tau, float tau2,
                                           bool two, float& F0, float& F1, float& F2, float& F0b) {
     for (int i = 0; i < n; ++i) {
-        const float z = sp.cz * st[i * BM + r];
-        const float x = z - tau;
+        const float a = st[i * BM + r];
+        const float x = fmaf(a, sp.cz, -tau);
         if (x > 0.f) add_sums<KIND>(x, sp.k, F0, F1, F2);
         if (two) {
-            const float x2 = z - tau2;
+            const float x2 = fmaf(a, sp.cz, -tau2);
             if (x2 > 0.f) F0b += pow_k<KIND>(x2, sp.k);
         }
     }
+}
+
+// Entries of one stash half above tau (z units): the row's support, when every candidate fit the stash.
+__device__ __forceinline__ uint32_t half_count(const float* st, int n, int r, float cz, float tau) {
+    uint32_t c = 0;
+    for (int i = 0; i < n; ++i) c += fmaf(st[i * BM + r], cz, -tau) > 0.f ? 1u : 0u;
+    return c;
 }
 
 __device__ __forceinline__ bool block_full(int J, int n, int causal, int row0) {
@@ -191,10 +207,15 @@ __device__ __forceinline__ bool block_full(int J, int n, int causal, int row0) {
     return last < n && (!causal || last <= row0);
 }
 
-template <int KIND>
+template <int KIND, int NB>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_h_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
+    using HC = HCfg<NB>;
+    constexpr int kHalf = HC::kHalf;
+    constexpr uint32_t offStash = HC::offStash;
+    constexpr uint32_t offV = HC::offV;
+    constexpr uint32_t offSmall = HC::offSmall;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = align_smem_1024(smem_raw);
     Small& sm = *reinterpret_cast<Small*>(smem + offSmall);
@@ -202,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* plan_bits = reinterpret_cast<uint32_t*>(&sm + 1);  // [2][W]
     uint32_t* next = plan_bits + 2 * W;                          // [W]
     uint32_t* mrow = next + W;                                   // [2][W]
-    uint32_t* live_all = mrow + 2 * W;                           // [128][kLiveStride]
+    uint32_t* live_all = mrow + 2 * W;                           // [128][HC::kStride]
     uint16_t* hist = reinterpret_cast<uint16_t*>(smem + offHist);
     float* stash = reinterpret_cast<float*>(smem + offStash);
 
@@ -221,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < NKS; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
         for (int i = 0; i < NVS; ++i) { mbar_init(&sm.v_full[i], 1); mbar_init(&sm.v_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
-            for (int b = 0; b < 2; ++b) {
+            for (int b = 0; b < NSB; ++b) {
                 mbar_init(&sm.s_full[i][b], 1);
                 mbar_init(&sm.s_empty[i][b], 4);
                 mbar_init(&sm.pv_free[i][b], 1);
@@ -299,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t sc0 = 0, sc1 = 0;    // per warpgroup: S tiles issued
             // per buffer (bit 2 g + b): parity of the commit of the P V that last read (or will read) it;
             // after k commits the barrier has completed phase k - 1, so the bits start at 1
-            uint32_t ppar = 0xfu;
+            uint32_t ppar = (1u << (2 * NSB)) - 1u;
             bool after_pv = false;
             int npv = 0;
             bool ok = wait_bounded(&sm.q_full, 0, abort_flag, a.status, true);
@@ -321,14 +342,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int ts = 0; ts < T && ok; ++ts) {
                     const int g = (kind == kSweepHist) ? 0 : (ts & 1);
                     const uint32_t sn = g ? sc1 : sc0;
-                    const uint32_t b = sn & 1u;
-                    const uint32_t bi = 2u * g + b;
+                    const uint32_t b = sn % NSB;
+                    const uint32_t bi = NSB * g + b;
                     const uint32_t ks = lc % NKS;
                     if (!(ok = wait_bounded(&sm.k_full[ks], (lc / NKS) & 1, abort_flag, a.status, true))) break;
-                    if (!(ok = wait_bounded(&sm.s_empty[g][b], ((sn >> 1) & 1) ^ 1, abort_flag, a.status, true))) break;
+                    if (!(ok = wait_bounded(&sm.s_empty[g][b], ((sn / NSB) & 1) ^ 1, abort_flag, a.status, true))) break;
                     if (pvk) {
-                        // the buffer last held block ts - 4 of this sweep: its P V must have completed
-                        if (ts >= 4 && !(ok = wait_bounded(&sm.pv_free[g][b], (ppar >> bi) & 1u, abort_flag, a.status, true)))
+                        // the buffer last held block ts - 2 NSB of this sweep: its P V must have completed
+                        if (ts >= 2 * NSB && !(ok = wait_bounded(&sm.pv_free[g][b], (ppar >> bi) & 1u, abort_flag, a.status, true)))
                             break;
                         ppar ^= 1u << bi;  // block ts's own P V, committed later by the P V thread
                     }
@@ -357,7 +378,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t idPV = idesc_f16_f32(BM, D, false, true);
             uint32_t vc = 0;              // V blocks consumed (ring order)
             uint32_t sc0 = 0, sc1 = 0;    // per warpgroup: S tiles issued (followed, not issued here)
-            uint32_t ppar = 0xfu;         // per buffer: parity of the last P V commit on its barrier
+            uint32_t ppar = (1u << (2 * NSB)) - 1u;  // per buffer: parity of the last P V commit on its barrier
             bool ok = true;
             for (int sw = 0; ok; ++sw) {
                 if (!(ok = wait_bounded(&sm.ctrl, sw & 1, abort_flag, a.status, true))) break;
@@ -375,8 +396,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int tp = 0; tp < T && ok; ++tp) {
                     const int g = tp & 1;
                     const uint32_t sn = g ? sc1 : sc0;
-                    const uint32_t b = sn & 1u;
-                    const uint32_t bi = 2u * g + b;
+                    const uint32_t b = sn % NSB;
+                    const uint32_t bi = NSB * g + b;
                     const uint32_t vs = vc % NVS;
                     // k P V products on a buffer so far: its P / U store number k + 1 completes phase k
                     if (!(ok = wait_bounded(&sm.pu_full[g][b], ((ppar >> bi) & 1u) ^ 1u, abort_flag, a.status, true))) break;
@@ -390,7 +411,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t acc = (tp == 0 && kk == 0) ? 0u : 1u;
                         mma_ts(tmem + kColO, tpu + 8 * kk, dv, idPV, acc);
                         mma_ts(tmem + kColOb, tpu + 32 + 8 * kk, dv, idPV, acc);
-                        mma_ts(tmem + kColOb, tmem + kColUlo + 32u * bi + 8 * kk, dv, idPV, 1u);
                     }
                     mma_commit(&sm.pv_free[g][b]);
                     mma_commit(&sm.v_empty[vs]);
@@ -441,18 +461,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         uint32_t sc = 0, pc = 0;
         uint32_t colS = 0;  // TMEM column of the S tile loaded last
+        uint32_t curb = 0;  // its buffer index
         int sw = 0;
         bool ok = true;
         float vbuf[BN];
 
         auto load_S = [&]() -> bool {
-            const uint32_t sb = sc & 1;
-            const bool got = wait_bounded(&sm.s_full[g][sb], (sc >> 1) & 1, abort_flag, a.status);
+            const uint32_t sb = sc % NSB;
+            const bool got = wait_bounded(&sm.s_full[g][sb], (sc / NSB) & 1, abort_flag, a.status);
             if (!__all_sync(0xffffffffu, got)) return false;
             tc_fence_after();
             __syncwarp();
             uint32_t* rr = reinterpret_cast<uint32_t*>(vbuf);
-            colS = 64u * (2u * g + sb);
+            colS = 64u * (NSB * g + sb);
+            curb = sb;
             tmem_ld32(lane_base + colS, rr);
             tmem_ld32(lane_base + colS + 32, rr + 32);
             tmem_ld_wait();
@@ -523,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const bool room = fl && nst > kHalf - 8;
                         if (__any_sync(0xffffffffu, room)) {
                             if (room) {
-                                nst = stash_prune(nst, st_mine, r, thr);
+                                nst = stash_prune(nst, st_mine, r, thr, kHalf);
                                 if (nst < 0) { ovf = true; nst = 0; }
                             }
                             fl = fl && !ovf;
@@ -549,10 +571,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         RowSolve s;
         bool row_ovf = false;
         float Su_stash = 0.f;
+        uint32_t nsup = 0;  // the row's support size (warpgroup 0)
         float m_raw = -INFINITY;
         int n1 = 0;
         if (g == 0) {
-            hist_init(h, live_all, r);
+            hist_init(h, live_all, r, HC::kStride);
             const int c1 = __float_as_int(sm.xf[kXCnt1][r]);
             m_raw = fmaxf(m_run, sm.xf[kXMax1][r]);
             row_ovf = ovf || c1 < 0;
@@ -581,6 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 half_sums<KIND>(st_mine, nst, r, sp, s.tau, s.tau, false, F0, F1, F2, F0b);
                 half_sums<KIND>(stash + kHalf * BM, n1, r, sp, s.tau, s.tau, false, F0, F1, F2, F0b);
                 Su_stash = F1;
+                nsup = half_count(st_mine, nst, r, sp.cz, s.tau) + half_count(stash + kHalf * BM, n1, r, sp.cz, s.tau);
             }
             sm.xf[kXOvf][r] = (valid && row_ovf) ? 1.0f : 0.0f;
         }
@@ -654,14 +678,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mask_S(J);
                     const float amax = group_max();
                     const bool keep = sp.cz * amax > lo0;
-                    if (sp.cz * amax - t > 0.f) {
+                    if (fmaf(amax, sp.cz, -t) > 0.f) {
 #pragma unroll
                         for (int q = 0; q < 8; ++q) {
-                            if (sp.cz * gm[q] - t > 0.f) {
+                            if (fmaf(gm[q], sp.cz, -t) > 0.f) {
 #pragma unroll
                                 for (int e = 0; e < 8; ++e) {
-                                    const float z = sp.cz * vbuf[8 * q + e];
-                                    const float x = z - t;
+                                    const float x = fmaf(vbuf[8 * q + e], sp.cz, -t);
                                     if constexpr (KIND == kAlpha15) {
                                         const float xp = fmaxf(x, 0.f);
                                         F0 = fmaf(xp, xp, F0);
@@ -674,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         if (x > 0.f) add_sums<KIND>(x, sp.k, F0, F1, F2);
                                     }
                                     if (two) {
-                                        const float x2 = z - t2;
+                                        const float x2 = fmaf(vbuf[8 * q + e], sp.cz, -t2);
                                         if (x2 > 0.f) F0b += pow_k<KIND>(x2, sp.k);
                                     }
                                 }
@@ -715,6 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float t = sm.xf[kXTau][r], lo0 = sm.xf[kXLo][r];
             const bool need_sums = __any_sync(0xffffffffu, sm.xf[kXOvf][r] != 0.0f);
             float Sp = 0.f, Sq = 0.f, F2 = 0.f;
+            uint32_t Sn = 0;
             const uint32_t* bits_p = plan_bits + (sw & 1) * W;
             int p = 0;
             for (int wd = 0; wd < W && ok; ++wd) {
@@ -727,7 +751,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mask_S(J);
                     const float amax = group_max();
                     const bool keep = sp.cz * amax > lo0;
-                    const bool nz = sp.cz * amax - t > 0.f;
+                    const bool nz = fmaf(amax, sp.cz, -t) > 0.f;
                     // two branch-free passes over the block, P then U, through one 32-word array; the solver
                     // sums ride on the P pass, in warps that hold a row whose tau still needs the check
                     uint32_t w32[32];
@@ -738,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             float p2[2];
 #pragma unroll
                             for (int h2 = 0; h2 < 2; ++h2) {
-                                const float x = sp.cz * vbuf[c + h2] - t;
+                                const float x = fmaf(vbuf[c + h2], sp.cz, -t);
                                 float pp, uu;
                                 if constexpr (KIND == kAlpha15) {
                                     uu = fmaxf(x, 0.f);
@@ -758,6 +782,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 if constexpr (SUMS) {
                                     Sp += pp;
                                     Sq += uu;
+                                    Sn += x > 0.f ? 1u : 0u;
                                 }
                                 p2[h2] = pp;
                             }
@@ -769,17 +794,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // P and U go into the columns of the S tile just read (this warpgroup's own buffer)
                     const uint32_t tp = lane_base + colS;
                     tmem_st32(tp, w32);
-                    // U = hi + lo: hi next to P, lo into the buffer paired with this S buffer (free for the
-                    // same reason: this S tile was issued after the P V that read the old contents)
+                    // U next to P, one fp16 term, in two halves of 32 keys
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        uint32_t whi[16], wlo[16];
+                        uint32_t wu[16];
 #pragma unroll
                         for (int c = 0; c < 32; c += 2) {
                             float u2[2];
 #pragma unroll
                             for (int h2 = 0; h2 < 2; ++h2) {
-                                const float x = sp.cz * vbuf[32 * h + c + h2] - t;
+                                const float x = fmaf(vbuf[32 * h + c + h2], sp.cz, -t);
                                 if constexpr (KIND == kAlpha15) {
                                     u2[h2] = fmaxf(x, 0.f);
                                 } else if constexpr (KIND == kAlpha2) {
@@ -790,18 +814,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     u2[h2] = pos ? exp2f((sp.k - 1.f) * __log2f(xs)) : 0.f;
                                 }
                             }
-                            const __half2 hh = __floats2half2_rn(u2[0], u2[1]);
-                            const float2 hf = __half22float2(hh);
-                            whi[c / 2] = *reinterpret_cast<const uint32_t*>(&hh);
-                            wlo[c / 2] = pack_half2(u2[0] - hf.x, u2[1] - hf.y);
+                            wu[c / 2] = pack_half2(u2[0], u2[1]);
                         }
-                        tmem_st16(tp + 32 + 16 * h, whi);
-                        tmem_st16(lane_base + kColUlo + (colS >> 1) + 16 * h, wlo);
+                        tmem_st16(tp + 32 + 16 * h, wu);
                     }
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&sm.pu_full[g][(colS >> 6) & 1u]);
+                    if (lane == 0) mbar_arrive(&sm.pu_full[g][curb]);
                     ++pc;
                     const uint32_t kb = __ballot_sync(0xffffffffu, keep);
                     const uint32_t nb = __ballot_sync(0xffffffffu, nz);
@@ -815,6 +835,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 sm.xf[kXF0][r] = Sp;
                 sm.xf[kXF1][r] = Sq;
                 sm.xf[kXF2][r] = F2;
+                sm.xf[kXCnt][r] = __uint_as_float(Sn);
             }
             ++pv;
             ok = !bar_or256(!ok || *abort_flag != 0);
@@ -824,6 +845,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     Sp += sm.xf[kXF0][r];
                     Su = Sq + sm.xf[kXF1][r];
                     F2 += sm.xf[kXF2][r];
+                    nsup = Sn + __float_as_uint(sm.xf[kXCnt][r]);
                     const float before = s.tau;
                     solve_step(s, Sp, Su, F2, 0.f, sp);
                     changed = s.tau != before;
@@ -907,6 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (g == 0 && valid) {
                 if (row_ovf) atomicAdd(&sm.st.overflow_rows, 1u);
                 atomicAdd(&sm.st.rows, 1u);
+                atomicAdd(&sm.st.support, nsup);
                 atomicAdd(&sm.st.steps, (uint32_t)s.steps);
                 atomicAdd(&sm.st.fallbacks, (uint32_t)s.fallbacks);
                 atomicAdd(&sm.st.step_hist[min(s.steps, kMaxSteps)], 1u);
@@ -914,6 +937,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             named_bar_sync(1, kCompute);
             if (tid == 0) {
                 sm.st.sweeps = (uint32_t)(1 + refine + pv);
+                sm.st.causal_blocks = tile_causal_blocks(2 * qt, 2, a.nqb, a.nkb, a.causal);
                 flush_stats(a.stats, sm.st);
             }
         }
@@ -927,34 +951,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int KIND>
+template <int KIND, int NB>
 cudaError_t launch_fwd_h_t(const FwdArgs& a, cudaStream_t stream) {
     CUtensorMap tq, tk, tv;
     cudaError_t e;
     if ((e = make_tmap_f16(&tq, a.Qh, a.B * a.H, a.n, D, BM)) != cudaSuccess) return e;
     if ((e = make_tmap_f16(&tk, a.Kh, a.B * a.H, a.n, D, BN)) != cudaSuccess) return e;
     if ((e = make_tmap_f16(&tv, a.Vh, a.B * a.H, a.n, D, BN)) != cudaSuccess) return e;
-    const size_t bytes = fwd_h_smem_bytes(a.nw);
+    const size_t bytes = fwd_h_smem_bytes(a.nw, NB);
     if (bytes > 232448) return cudaErrorInvalidConfiguration;
-    auto kern = fwd_h_kernel<KIND>;
+    auto kern = fwd_h_kernel<KIND, NB>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
         return e;
     dim3 grid(a.ntiles, a.B * a.H);
+    launch_mark(stream);
     kern<<<grid, kThreads, bytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError();
 }
 
+template <int NB>
+cudaError_t launch_fwd_h_nb(const FwdArgs& a, cudaStream_t stream) {
+    if (a.sp.alpha == 1.5f) return launch_fwd_h_t<kAlpha15, NB>(a, stream);
+    if (a.sp.alpha == 2.0f) return launch_fwd_h_t<kAlpha2, NB>(a, stream);
+    return launch_fwd_h_t<kGeneric, NB>(a, stream);
+}
+
 }  // namespace
 
-size_t fwd_h_smem_bytes(int nw) {
-    return 1024 + offSmall + sizeof(Small) + (size_t)5 * nw * 4 + (size_t)BM * kLiveStride * 4;
+size_t fwd_h_smem_bytes(int nw, int bins) {
+    if (bins > 256) {
+        using HC = HCfg<512>;
+        return 1024 + HC::offSmall + sizeof(Small) + (size_t)5 * nw * 4 + (size_t)BM * HC::kStride * 4;
+    }
+    using HC = HCfg<256>;
+    return 1024 + HC::offSmall + sizeof(Small) + (size_t)5 * nw * 4 + (size_t)BM * HC::kStride * 4;
 }
 
 cudaError_t launch_fwd_h(const FwdArgs& a, cudaStream_t stream) {
     if (a.d != 64 || !(a.sp.alpha <= 2.0f)) return cudaErrorInvalidValue;
-    if (a.sp.alpha == 1.5f) return launch_fwd_h_t<kAlpha15>(a, stream);
-    if (a.sp.alpha == 2.0f) return launch_fwd_h_t<kAlpha2>(a, stream);
-    return launch_fwd_h_t<kGeneric>(a, stream);
+    if (a.sp.bins > 256) return launch_fwd_h_nb<512>(a, stream);
+    return launch_fwd_h_nb<256>(a, stream);
 }
 
 }  // namespace eattn

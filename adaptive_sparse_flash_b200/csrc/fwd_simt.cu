@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "fwd_common.cuh"
+#include "launch.h"
 
 namespace eattn {
 namespace {
@@ -199,6 +200,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
 
     // ---- P V sweep: O, U V, sum u, exact mask; the sums double as the check of sum p = 1 ----
     float Su = 0.f;
+    uint32_t nsup = 0;  // nonzero probabilities of this row in the last P V sweep
     auto pv_sweep = [&]() -> bool {
         __syncthreads();
         for (int i = tid; i < cwords; i += blockDim.x) next[i] = 0u;
@@ -207,6 +209,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
         __syncthreads();
         float Sp = 0.f, F2 = 0.f;
         Su = 0.f;
+        nsup = 0;
         const float t = s.tau, lo0 = s.lo;
         for (int wd = 0; wd < cwords; ++wd) {
             uint32_t bits = cand[wd];
@@ -231,6 +234,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
                         else { u = exp2f((sp.k - 1.f) * __log2f(x)); p = u * x; F2 += __fdividef(u, x); }
                         Sp += p;
                         Su += u;
+                        ++nsup;
                         nz = true;
                         const float* v = sV + jj * D;
                         for (int c = 0; c < D; ++c) {
@@ -279,6 +283,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
         if (a.steps) a.steps[head + row] = (uint8_t)s.steps;
         if (sh.overflow) atomicAdd(&st.overflow_rows, 1u);
         atomicAdd(&st.rows, 1u);
+        atomicAdd(&st.support, nsup);
         atomicAdd(&st.steps, (uint32_t)s.steps);
         atomicAdd(&st.fallbacks, (uint32_t)s.fallbacks);
         atomicAdd(&st.step_hist[min(s.steps, kMaxSteps)], 1u);
@@ -295,6 +300,7 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
         __syncthreads();
         if (tid == 0) {
             st.sweeps = (uint32_t)sweeps;
+            st.causal_blocks = tile_causal_blocks(qb0, mrows, a.nqb, a.nkb, a.causal);
             flush_stats(a.stats, st);
         }
     }
@@ -311,6 +317,7 @@ cudaError_t launch_t(const FwdArgs& a, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
     dim3 grid(a.ntiles, a.B * a.H);
+    launch_mark(stream);
     kern<<<grid, 128, bytes, stream>>>(a);
     return cudaGetLastError();
 }

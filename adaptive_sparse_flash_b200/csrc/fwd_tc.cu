@@ -551,10 +551,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // ---- P V sweep: p, u to shared memory for the P V / U V MMAs, exact mask, sum check ----
         float Su = 0.f;
+        uint32_t nsup = 0;  // nonzero probabilities of this row in the last P V sweep
         auto pv_sweep = [&]() -> bool {
             publish(kSweepPV);
             float Sp = 0.f, F2 = 0.f;
             Su = 0.f;
+            nsup = 0;
             const float t = s.tau, lo0 = s.lo;
             const uint32_t* bits_p = plan_bits + (sw & 1) * W;
             for (int wd = 0; wd < W && ok; ++wd) {
@@ -608,6 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         }
                                         Sp += p;
                                         Su += u;
+                                        nsup += x > 0.f ? 1u : 0u;
                                         pv2[q] = p;
                                         uv2[q] = u;
                                     }
@@ -720,6 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (valid) {
                 if (sh.overflow) atomicAdd(&sm.st.overflow_rows, 1u);
                 atomicAdd(&sm.st.rows, 1u);
+                atomicAdd(&sm.st.support, nsup);
                 atomicAdd(&sm.st.steps, (uint32_t)s.steps);
                 atomicAdd(&sm.st.fallbacks, (uint32_t)s.fallbacks);
                 atomicAdd(&sm.st.step_hist[min(s.steps, kMaxSteps)], 1u);
@@ -727,6 +731,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             named_bar_sync(1, BM);
             if (r == 0) {
                 sm.st.sweeps = (uint32_t)(1 + refine + pv);
+                sm.st.causal_blocks = tile_causal_blocks(2 * qt, 2, a.nqb, a.nkb, a.causal);
                 flush_stats(a.stats, sm.st);
             }
         }
@@ -802,6 +807,7 @@ static cudaError_t launch_fwd_tc_t(const FwdArgs& a, cudaStream_t stream) {
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
         return e;
     dim3 grid(a.ntiles, a.B * a.H);
+    launch_mark(stream);
     kern<<<grid, kThreads, bytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError();
 }

@@ -9,6 +9,10 @@
 
 namespace eattn {
 
+// Records the caller's next timing event (entmax_opts.events) on `stream`, if the current API call was given
+// any; every launcher calls it right before each kernel launch (api.cu).
+void launch_mark(cudaStream_t stream);
+
 // fp16 operand copies (f16.cu): `count` bf16 tensors of n16 16-byte chunks each; maxbits[t] receives
 // max |x| of tensor t as float bits.
 struct F16Job {
@@ -29,7 +33,7 @@ __host__ __device__ inline int f16_range_exp(uint32_t maxbits) {
 
 cudaError_t launch_fwd_simt(const FwdArgs& a, bool fp32, cudaStream_t stream);
 cudaError_t launch_fwd_h(const FwdArgs& a, cudaStream_t stream);
-size_t fwd_h_smem_bytes(int nw);
+size_t fwd_h_smem_bytes(int nw, int bins);
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t stream);
 size_t fwd_tc_smem_bytes(int d, int nw);
 size_t fwd_simt_smem_bytes(int d, int nkb, int mb, int nw);

@@ -33,6 +33,7 @@ cudaError_t launch_mask_transpose(const uint32_t* mask, uint32_t* maskT, int BH,
                                   cudaStream_t stream) {
     const int words = nkb * nwq;
     dim3 grid((words + 255) / 256, BH);
+    launch_mark(stream);
     mask_transpose_kernel<<<grid, 256, 0, stream>>>(mask, maskT, nqb, nkb, nw, nwq);
     return cudaGetLastError();
 }

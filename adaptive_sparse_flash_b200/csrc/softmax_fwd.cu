@@ -280,6 +280,7 @@ cudaError_t launch_t(const SoftmaxFwdArgs& a, cudaStream_t stream) {
     auto kern = softmax_fwd_kernel<D>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
         return e;
+    launch_mark(stream);
     kern<<<dim3(a.ntiles, BH), kThreads, bytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError();
 }

@@ -352,6 +352,7 @@ cudaError_t launch_softmax_fwd_h(const SoftmaxFwdArgs& a, cudaStream_t stream) {
         cudaSuccess)
         return e;
     dim3 grid(a.ntiles, a.B * a.H);
+    launch_mark(stream);
     softmax_fwd_h_kernel<<<grid, kThreads, bytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError();
 }

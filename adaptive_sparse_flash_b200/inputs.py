@@ -23,6 +23,7 @@ __all__ = [
     "iid",
     "clustered",
     "sample_rows",
+    "sample_blocks",
 ]
 
 
@@ -121,3 +122,21 @@ def sample_rows(n: int, count: int, *, seed: int = 0) -> np.ndarray:
     picks = rng.choice(n, size=count, replace=False)
     picks = np.unique(np.concatenate([picks, [0, n - 1]]))
     return picks.astype(np.int64)
+
+
+def sample_blocks(n: int, block: int, count: int, *, seed: int = 0) -> np.ndarray:
+    """Every row of `count` distinct whole query blocks of `block` rows, drawn from default_rng(seed + 1).
+
+    Always includes the first and the last block (the first causal rows and the ragged tail). Sampling whole
+    blocks lets a test check the block mask rows of the sample exactly, in both directions.
+    """
+    rng = np.random.default_rng(seed + 1)
+    nb = (n + block - 1) // block
+    count = min(count, nb)
+    picks = rng.choice(nb, size=count, replace=False)
+    picks = np.unique(np.concatenate([picks, [0, nb - 1]]))
+    if len(picks) > count:  # keep the two ends, drop interior picks beyond the count
+        inner = picks[(picks != 0) & (picks != nb - 1)][: max(0, count - 2)]
+        picks = np.unique(np.concatenate([inner, [0, nb - 1]]))
+    rows = (picks[:, None] * block + np.arange(block)[None, :]).ravel()
+    return rows[rows < n].astype(np.int64)

@@ -70,6 +70,7 @@ typedef struct {
     unsigned long long nonzero_blocks;   /* mask bits set                                         */
     unsigned long long sweeps;           /* key sweeps over all tiles (dense + refine + P V)      */
     unsigned long long overflow_rows;    /* rows whose candidates did not fit the on-chip stash   */
+    unsigned long long support;          /* nonzero probabilities (entries with z > tau), all rows */
 } entmax_stats;
 
 typedef struct {
@@ -82,7 +83,24 @@ typedef struct {
     entmax_stats* stats;    /* optional device counters, may be NULL                               */
     float* tau_hist;        /* optional device [B,H,n]: the histogram bound tau_h of each row      */
     uint8_t* steps;         /* optional device [B,H,n]: solver steps taken by each row             */
+    void* const* events;    /* optional cudaEvent_t handles (as void*) for per-kernel timing, or NULL */
+    int num_events;         /* length of `events` (0 when NULL); see "Per-kernel timing" below       */
 } entmax_opts;
+
+/* Per-kernel timing. When opts->events is set, a call records events[i] on `stream` right before its i-th
+ * kernel launch and one more event after its last launch (events past num_events are not recorded; a NULL
+ * handle is skipped). The launches of a call, in order:
+ *   entmax_attn_fwd, bf16, d = 64, alpha <= 2:  to_f16_pass1, to_f16_pass2, fwd_h, mask_transpose
+ *   entmax_attn_fwd, bf16, otherwise:           fwd_tc, mask_transpose
+ *   entmax_attn_fwd, fp32:                      fwd_simt
+ *   entmax_attn_bwd, d = 64, alpha <= 2:        to_f16_pass1, to_f16_pass2, bwd_pre, bwd_h_dq, bwd_h_dkdv
+ *   entmax_attn_bwd, otherwise:                 bwd_pre, bwd_dkdv, bwd_dq
+ *   softmax_attn_fwd, d = 64 with a workspace:  to_f16_pass1, to_f16_pass2, softmax_fwd_h
+ *   softmax_attn_fwd, otherwise:                softmax_fwd
+ *   softmax_attn_bwd, d = 64:                   to_f16_pass1, to_f16_pass2, bwd_pre, bwd_h_dq, bwd_h_dkdv
+ *   softmax_attn_bwd, d = 128:                  bwd_pre, bwd_dkdv, bwd_dq
+ * The events are recorded by the host thread that makes the call, as part of it; opts->events must stay
+ * valid for the duration of the call only. */
 
 /* Bytes of workspace that entmax_attn_fwd/bwd (or softmax_attn_fwd/bwd) need for these sizes.
  * Returns 0 for invalid sizes. opts may be NULL (defaults). */
@@ -131,7 +149,9 @@ entmax_status softmax_attn_bwd(const void* Q, const void* K, const void* V, cons
  * each device looks up the array's device address (cudaGetSymbolAddress), so make that first call
  * before any stream capture. All calls share the array and it keeps the last call's contents (no part
  * of it needs to start at zero); calls that may overlap on the GPU (other streams, other host threads)
- * race on it, and a later entmax_attn_bwd cannot use it: for training use entmax_attn_fwd. */
+ * race on it, and a later entmax_attn_bwd cannot use it: for training use entmax_attn_fwd. The looked-up address
+ * is kept for the life of the process: do not use this entry point after cudaDeviceReset() on that device (the
+ * same holds for the device status word behind every entry point). */
 entmax_status entmax_attn_fwd_noalloc(const void* Q, const void* K, const void* V, void* O, float* tau,
                                       uint32_t* block_mask, int B, int H, int n, int d, float alpha, int causal,
                                       entmax_dtype dt, const entmax_opts* opts, void* stream);
@@ -148,7 +168,7 @@ entmax_status entmax_attn_selftest_timeout(int limit_us, void* stream);
 /* Human-readable name of a status code (static string). */
 const char* entmax_status_str(entmax_status s);
 
-/* Library ABI version: 1. */
+/* Library ABI version: 2 (entmax_opts gained `events` and `num_events`). */
 int entmax_attn_version(void);
 
 #ifdef __cplusplus

@@ -130,6 +130,7 @@ def forward(Q, K, V, alpha, causal, scale=None, block=64, rows=None, chunk=256):
     sum_u = np.zeros((B, H, r))
     row_bits = np.zeros((B, H, r, nkb), dtype=bool)
     row_bmax = np.zeros((B, H, r, nkb))
+    support = np.zeros((B, H, r), dtype=np.int64)
     for b in range(B):
         for h in range(H):
             for c0 in range(0, r, chunk):
@@ -144,8 +145,9 @@ def forward(Q, K, V, alpha, causal, scale=None, block=64, rows=None, chunk=256):
                 np.maximum.at(bm, (res["rr"], res["cc"] // block), res["p_s"])
                 row_bmax[b, h, sl] = bm
                 row_bits[b, h, sl] = bm > 0.0
+                support[b, h, sl] = np.bincount(res["rr"], minlength=len(sel))
     out = dict(O=O, Obar=Obar, tau=tau, sum_u=sum_u, row_bits=row_bits, row_bmax=row_bmax,
-               rows=rows, scale=scale)
+               support=support, rows=rows, scale=scale)
     if full:
         nqb = (n + block - 1) // block
         padb = np.zeros((B, H, nqb * block, nkb), dtype=bool)

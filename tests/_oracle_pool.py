@@ -32,6 +32,12 @@ def _head_job(args):
     if kind == "bwd_full":
         dQ, dK, dV = oa.backward(Q, K, V, do[None, None], alpha, causal, key_cols=cols)
         return dQ[0, 0], dK[0, 0], dV[0, 0]
+    if kind == "sens":
+        tests = os.path.dirname(os.path.abspath(__file__))
+        if tests not in sys.path:
+            sys.path.insert(0, tests)
+        from _parity import grad_sensitivity
+        return grad_sensitivity(q, k, v, do, alpha, causal)
     raise ValueError(kind)
 
 

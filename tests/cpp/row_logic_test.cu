@@ -20,10 +20,13 @@ template <int KIND> int run(double k, float alpha) {
   int bad = 0;
   srand(3);
   for (int trial = 0; trial < 3000; ++trial) {
-    const int B = (trial % 3 == 0) ? 64 : 256;
-    std::vector<uint16_t> hist(256 * 128, 0);
-    uint32_t live[9] = {0};
-    HistRow h; h.live = live; h.top = 1000 + rand() % 500; h.any = true;
+    const int B = (trial % 4 == 0) ? 64 : (trial % 4 == 1) ? 512 : (trial % 4 == 2) ? 128 : 256;
+    std::vector<uint16_t> hist(512 * 128, 0);
+    uint32_t live_all[6 * 17] = {0};
+    HistRow h;
+    hist_init(h, live_all, 5, B > 256 ? kLiveStride512 : kLiveStride);
+    uint32_t* live = h.live;
+    h.top = 1000 + rand() % 500; h.any = true;
     std::vector<int> c(B, 0);
     c[0] = 1 + rand() % 3;
     const int nb = rand() % 40;
@@ -33,7 +36,7 @@ template <int KIND> int run(double k, float alpha) {
     // some dead slots with garbage counts
     for (int i = 0; i < 5; ++i) { int j = rand() % B; if (!c[j]) { int sl = (h.top - j) & (B - 1); hist[sl * 128 + r] = 77; } }
     SolveParams sp = make_solve_params(alpha, 0.125f, B, 0);
-    float T[260]; for (int i = 0; i <= B; ++i) T[i] = powf((float)i, sp.k);
+    float T[516]; for (int i = 0; i <= B; ++i) T[i] = powf((float)i, sp.k);
     const float got = hist_tau<KIND>(h, sp, hist.data(), r, T);
     const double ref = brute(c, h.top, B, k);
     const double tol = 1e-5 * fmax(1.0, fabs(ref)) + (KIND == kGeneric ? sp.w / 64 + 1e-5 : 0);
@@ -46,12 +49,12 @@ template <int KIND> int run(double k, float alpha) {
 }
 int ring_masks() {
   int bad = 0;
-  for (int B : {64, 128, 256})
+  for (int B : {64, 128, 256, 512})
     for (int s0 = 0; s0 < B; ++s0)
       for (int len = 0; len < B; ++len) {
-        uint32_t live[8];
-        for (int i = 0; i < 8; ++i) live[i] = 0xffffffffu & ~ring_word_mask(i, s0, len, B);
-        for (int p = 0; p < 256; ++p) {
+        uint32_t live[16];
+        for (int i = 0; i < 16; ++i) live[i] = 0xffffffffu & ~ring_word_mask(i, s0, len, B);
+        for (int p = 0; p < 512; ++p) {
           const bool cleared = p < B && ((p - s0) % B + B) % B < len;
           const bool bit = (live[p >> 5] >> (p & 31)) & 1u;
           if (bit == cleared) ++bad;

@@ -37,7 +37,7 @@ def test_library_exports_every_symbol(L):
 
 def test_version_and_status_strings(L):
     from adaptive_sparse_flash_b200 import binding as b
-    assert L.entmax_attn_version() == 1
+    assert L.entmax_attn_version() == 2
     for s in range(7):
         assert len(b.entmax_status_str(s)) > 0
     assert b.entmax_status_str(99) == "unknown status"
@@ -55,9 +55,11 @@ def test_workspace_size(L):
     assert b.entmax_attn_workspace_size(1, 1, 0, 64) == 0      # empty sequence
 
 
-def _fwd(L, ptr=16, n=64, d=64, alpha=1.5, causal=1, dt=0, ws=True, mask_block=0, bins=0, init_mode=0):
+def _fwd(L, ptr=16, n=64, d=64, alpha=1.5, causal=1, dt=0, ws=True, mask_block=0, bins=0, init_mode=0,
+         num_events=0):
     from adaptive_sparse_flash_b200 import binding as b
     o = b.EntmaxOpts()
+    o.num_events = num_events
     o.mask_block = mask_block
     o.hist_bins = bins
     o.init_mode = init_mode
@@ -83,6 +85,8 @@ def test_validation_errors_return_before_launch(L):
     assert _fwd(L, init_mode=5) == b.ENTMAX_ERR_INVALID
     assert _fwd(L, ptr=18) == b.ENTMAX_ERR_ALIGN
     assert _fwd(L, ws=False) == b.ENTMAX_ERR_WORKSPACE
+    assert _fwd(L, num_events=3) == b.ENTMAX_ERR_INVALID     # events count without an events array
+    assert _fwd(L, num_events=-1) == b.ENTMAX_ERR_INVALID
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

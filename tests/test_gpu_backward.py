@@ -6,7 +6,8 @@ from adaptive_sparse_flash_b200 import inputs
 from oracle import attention as oa
 from oracle import softmax as osm
 
-from _parity import BF16_MAX_ABS, BF16_MEAN_ABS, check_close, check_mask, check_tau, conditioning, to_torch
+from _parity import (BF16_MAX_ABS, BF16_MEAN_ABS, check_close, check_grads_bounded, check_mask, check_tau,
+                     grad_sensitivity, to_torch)
 
 pytestmark = pytest.mark.gpu
 
@@ -49,29 +50,36 @@ def test_bwd_small(torch_cuda, alpha, causal):
     _check_grads_conditioned(arr, alpha, causal, (dQ, dK, dV), (rdQ, rdK, rdV), f"bwd small a={alpha} c={causal}")
 
 
-# reading for alpha >= 2 (see _parity.conditioning): alpha = 2 rows with an entry within float32 rounding
-# of tau (flip), alpha > 2 rows with a support entry below 1e-2 are reported and left out of the gradient
-# comparison; alpha > 2 rows with a support entry below 1e-4 are left out of the O comparison.
-GRAD_FLIP = 2e-6
-GRAD_XMIN = "grad"  # per-row bound from _parity.grad_xmin
-FWD_XMIN = 1e-4
+# reading for alpha > 2 (see _parity.grad_sensitivity): u = x^(k-1) is unbounded at the support boundary, so
+# a gradient row with a support entry within float32 rounding of tau is not fixed by float32 scores. Every
+# row is still compared: within 2e-2 plus twice its derived bound, at most 2 % of all rows (of all heads)
+# over 2e-2, and the mean bound on the rows whose bound is below 2e-2. O and every alpha <= 2 gradient keep
+# the plain bounds on every row.
+GRAD_OVER_CAP = 0.02
 
 
-def _grad_conditioning(arr, alpha, causal):
-    if alpha > 2.0:
-        return conditioning(arr, alpha, causal, xmin=GRAD_XMIN)
-    return conditioning(arr, alpha, causal, xmin=0.0, flip=GRAD_FLIP)
-
-
-def _check_grads_conditioned(arr, alpha, causal, g, ref, where):
-    if alpha < 2.0:
+def _check_grads_conditioned(arr, alpha, causal, g, ref, where, cols=None):
+    if alpha <= 2.0:
         _check_grads(g, ref, where)
         return
-    bad_r, bad_c = _grad_conditioning(arr, alpha, causal)
-    print(f"{where}: ill-conditioned rows {bad_r.mean():.3f}, touched key columns {bad_c.mean():.3f}")
-    check_close(g[0][~bad_r], ref[0][~bad_r], BF16_MAX_ABS, BF16_MEAN_ABS, where + " dQ (conditioned rows)")
-    for name, x, y in zip(("dK", "dV"), g[1:], ref[1:]):
-        check_close(x[~bad_c], y[~bad_c], BF16_MAX_ABS, BF16_MEAN_ABS, f"{where} {name} (untouched columns)")
+    B, H = arr["Q"].shape[:2]
+    sens = [grad_sensitivity(arr["Q"][b, h], arr["K"][b, h], arr["V"][b, h], arr["dO"][b, h], alpha, causal)
+            for b in range(B) for h in range(H)]
+    _check_bounded_heads(g, ref, sens, H, cols, where)
+
+
+def _check_bounded_heads(g, ref, sens, H, cols, where):
+    tot = np.zeros((3, 3), np.int64)  # [dQ, dK, dV] x [over 2e-2, widened, rows]
+    for i, (sq, sk, sv) in enumerate(sens):
+        b, h = divmod(i, H)
+        if cols is not None:
+            sk, sv = sk[cols], sv[cols]
+        for t, (name, x, y, s) in enumerate(zip(("dQ", "dK", "dV"), g, ref, (sq, sk, sv))):
+            tot[t] += check_grads_bounded(x[b, h], y[b, h], s, f"{where} {name} (b={b}, h={h})")
+    for t, name in enumerate(("dQ", "dK", "dV")):
+        over, wide, rows = tot[t]
+        print(f"{where} {name}: {over / rows:.4f} of rows over 2e-2, {wide / rows:.4f} with a bound above 2e-2")
+        assert over <= GRAD_OVER_CAP * rows, f"{where} {name}: {over} of {rows} rows over 2e-2"
 
 
 @pytest.mark.parametrize("n", [1, 77, 200])
@@ -99,6 +107,11 @@ def test_cfg3_full(torch_cuda, beta):
     fw = per_head("fwd_rows", arr, 1.5, True, rows=rows)
     check_tau(tau, np.stack([r["tau"] for r in fw]).reshape(tau.shape), "cfg3 tau")
     check_close(O, np.stack([r["O"] for r in fw]).reshape(O.shape), BF16_MAX_ABS, BF16_MEAN_ABS, "cfg3 O")
+    # the d = 128 block mask, every block row: bit-exact except blocks whose oracle max p < 1e-3
+    nkb = 4096 // 64
+    r_bits = np.stack([r["row_bits"] for r in fw]).reshape(B, H, 64, 64, nkb).any(axis=3)
+    r_bmax = np.stack([r["row_bmax"] for r in fw]).reshape(B, H, 64, 64, nkb).max(axis=3)
+    check_mask(mask, r_bits, r_bmax, f"cfg3 beta={beta} mask")
 
 
 # ---- dense softmax baseline -----------------------------------------------------------------------------
@@ -128,25 +141,43 @@ def test_cfg4_sampled(torch_cuda):
     from _oracle_pool import per_head
     arr = inputs.clustered(1, 16, 16384, 64, centres=256, beta_q=6.0, seed=0)
     O, tau, mask, dQ, dK, dV = _fwd_bwd(torch_cuda, arr, 1.5, True)
-    rows = inputs.sample_rows(16384, 512, seed=0)
+    # 512 query rows per head as 8 whole 64-row blocks (first and last included), so that the mask rows of
+    # the sample are checked exactly in both directions; 512 seeded key columns for dK and dV
+    rows = inputs.sample_blocks(16384, 64, 8, seed=0)
     cols = inputs.sample_rows(16384, 512, seed=1)
+    assert len(rows) == 512
     fw = per_head("fwd_rows", arr, 1.5, True, rows=rows)
     check_tau(tau[:, :, rows], np.stack([r["tau"] for r in fw]).reshape(1, 16, -1), "cfg4 tau")
     check_close(O[:, :, rows], np.stack([r["O"] for r in fw]).reshape(1, 16, len(rows), 64),
                 BF16_MAX_ABS, BF16_MEAN_ABS, "cfg4 O")
-    from _parity import unpack_mask
     nkb = 256
-    g_bits = unpack_mask(mask, nkb)[:, :, rows // 64]          # the 64-row mask block of each sampled row
-    r_bits = np.stack([r["row_bits"] for r in fw]).reshape(1, 16, len(rows), nkb)
-    r_bmax = np.stack([r["row_bmax"] for r in fw]).reshape(1, 16, len(rows), nkb)
-    # a sampled row's nonzero blocks must be set in its block row (the block row may have more)
-    missing = r_bits & ~g_bits & (r_bmax >= 1e-3)
-    assert not missing.any(), f"cfg4 mask: {int(missing.sum())} nonzero blocks of sampled rows not set"
+    blocks = np.unique(rows // 64)
+    r_bits = np.stack([r["row_bits"] for r in fw]).reshape(1, 16, len(blocks), 64, nkb).any(axis=3)
+    r_bmax = np.stack([r["row_bmax"] for r in fw]).reshape(1, 16, len(blocks), 64, nkb).max(axis=3)
+    check_mask(mask[:, :, blocks], r_bits, r_bmax, "cfg4 mask (sampled block rows)")
     bw = per_head("bwd_full", arr, 1.5, True, cols=cols)
     rdQ = np.stack([r[0] for r in bw]).reshape(dQ.shape)
     rdK = np.stack([r[1] for r in bw]).reshape(1, 16, len(cols), 64)
     rdV = np.stack([r[2] for r in bw]).reshape(1, 16, len(cols), 64)
     _check_grads((dQ[:, :, rows], dK[:, :, cols], dV[:, :, cols]), (rdQ[:, :, rows], rdK, rdV), "cfg4")
+
+
+# ---- determinism: two calls give bit-identical outputs ---------------------------------------------------
+
+@pytest.mark.parametrize("alpha,d", [(1.5, 64), (2.0, 64), (1.5, 128), (3.0, 64)])
+def test_determinism(torch_cuda, alpha, d):
+    from adaptive_sparse_flash_b200 import binding as b
+    arr = inputs.clustered(2, 3, 1100, d, centres=16, beta_q=4.0, seed=17)
+    t = to_torch(arr, torch_cuda.bfloat16)
+    outs = []
+    for _ in range(2):
+        f = b.forward(t["Q"], t["K"], t["V"], alpha, True)
+        dQ, dK, dV = b.backward(t["Q"], t["K"], t["V"], f, t["dO"])
+        torch_cuda.cuda.synchronize()
+        outs.append((f.O, f.tau, f.mask, dQ, dK, dV))
+    assert b.entmax_attn_check() == 0
+    for name, x, y in zip(("O", "tau", "mask", "dQ", "dK", "dV"), *outs):
+        assert torch_cuda.equal(x, y), f"{name} differs between two identical calls"
 
 
 # ---- configuration 5: 8 x 12 x 2048 x 64 alpha sweep, every solver branch ------------------------------
@@ -171,23 +202,13 @@ def test_cfg5_alpha_sweep(torch_cuda, alpha, beta):
     fw = per_head("fwd_rows", arr, alpha, True, rows=rows)
     O, tau = f.O.float().cpu().numpy(), f.tau.cpu().numpy()
     check_tau(tau, np.stack([r["tau"] for r in fw]).reshape(tau.shape), "cfg5 tau")
-    rO = np.stack([r["O"] for r in fw]).reshape(O.shape)
-    if alpha > 2.0:
-        bad_o, _ = conditioning(arr, alpha, True, xmin=FWD_XMIN)
-        print(f"cfg5 a={alpha} b={beta}: O rows with a support entry below {FWD_XMIN}: {bad_o.mean():.4f}")
-        check_close(O[~bad_o], rO[~bad_o], BF16_MAX_ABS, BF16_MEAN_ABS, "cfg5 O (conditioned rows)")
-    else:
-        check_close(O, rO, BF16_MAX_ABS, BF16_MEAN_ABS, "cfg5 O")
+    check_close(O, np.stack([r["O"] for r in fw]).reshape(O.shape), BF16_MAX_ABS, BF16_MEAN_ABS, "cfg5 O")
     rdQ = np.stack([r[0] for r in bw]).reshape(dQ.shape)
     rdK = np.stack([r[1] for r in bw]).reshape(8, 12, len(cols), 64)
     rdV = np.stack([r[2] for r in bw]).reshape(8, 12, len(cols), 64)
     g = (dQ.cpu().numpy(), dK.cpu().numpy()[:, :, cols], dV.cpu().numpy()[:, :, cols])
-    if alpha < 2.0:
+    if alpha <= 2.0:
         _check_grads(g, (rdQ, rdK, rdV), f"cfg5 a={alpha} b={beta}")
     else:
-        bad_r, bad_c = _grad_conditioning(arr, alpha, True)
-        bad_c = bad_c[:, :, cols]
-        print(f"cfg5 a={alpha} b={beta}: ill-conditioned rows {bad_r.mean():.3f}, columns {bad_c.mean():.3f}")
-        check_close(g[0][~bad_r], rdQ[~bad_r], BF16_MAX_ABS, BF16_MEAN_ABS, "cfg5 dQ (conditioned rows)")
-        check_close(g[1][~bad_c], rdK[~bad_c], BF16_MAX_ABS, BF16_MEAN_ABS, "cfg5 dK (untouched columns)")
-        check_close(g[2][~bad_c], rdV[~bad_c], BF16_MAX_ABS, BF16_MEAN_ABS, "cfg5 dV (untouched columns)")
+        sens = per_head("sens", arr, alpha, True)
+        _check_bounded_heads(g, (rdQ, rdK, rdV), sens, 12, cols, f"cfg5 a={alpha} b={beta}")

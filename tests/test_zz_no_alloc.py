@@ -10,7 +10,7 @@ import pytest
 
 from adaptive_sparse_flash_b200 import inputs
 
-from _parity import BF16_MAX_ABS, BF16_MEAN_ABS, TAU_REL, to_torch
+from _parity import to_torch
 
 pytestmark = pytest.mark.gpu
 
@@ -58,11 +58,10 @@ def test_noalloc_forward_matches_workspace_forward(env):
         assert st == b.ENTMAX_OK, b.entmax_status_str(st)
         torch.cuda.synchronize()
         assert b.entmax_attn_check() == 0
+        # the same kernels on the same inputs: identical outputs, whichever memory holds the scratch
         O = O1.float().cpu().numpy()
-        diff = np.abs(O - ref[0])
-        assert diff.max() <= BF16_MAX_ABS and diff.mean() <= BF16_MEAN_ABS, (call, diff.max())
-        rel = np.abs(tau1.cpu().numpy() - ref[1]) / np.maximum(1.0, np.abs(ref[1]))
-        assert rel.max() <= TAU_REL, (call, rel.max())
+        assert np.array_equal(O, ref[0]), (call, float(np.abs(O - ref[0]).max()))
+        assert np.array_equal(tau1.cpu().numpy(), ref[1]), call
         assert np.array_equal(mask1.cpu().numpy(), ref[2]), call
 
 
