@@ -37,6 +37,8 @@ EXPORTS = (
     "entmax_status_str",
     "entmax_attn_version",
     "entmax_attn_fwd_noalloc",
+    "entmax_attn_saved_size",
+    "entmax_attn_scratch_size",
 )
 
 
@@ -77,6 +79,8 @@ class EntmaxOpts(ctypes.Structure):
         ("steps", ctypes.c_void_p),
         ("events", ctypes.c_void_p),
         ("num_events", ctypes.c_int),
+        ("scratch", ctypes.c_void_p),
+        ("scratch_bytes", ctypes.c_size_t),
     ]
 
 
@@ -95,8 +99,9 @@ def lib() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     op = ctypes.POINTER(EntmaxOpts)
-    L.entmax_attn_workspace_size.argtypes = [i, i, i, i, i, op]
-    L.entmax_attn_workspace_size.restype = sz
+    for nm in ("entmax_attn_workspace_size", "entmax_attn_saved_size", "entmax_attn_scratch_size"):
+        getattr(L, nm).argtypes = [i, i, i, i, i, op]
+        getattr(L, nm).restype = sz
     L.entmax_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, op, vp]
     L.entmax_attn_fwd.restype = i
     L.entmax_attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, op, vp]
@@ -150,7 +155,7 @@ def _dtype_code(t) -> int:
 
 
 def make_opts(workspace=None, *, scale=0.0, mask_block=0, hist_bins=0, init_mode=0,
-              stats=None, tau_hist=None, steps=None, events=None) -> EntmaxOpts:
+              stats=None, tau_hist=None, steps=None, events=None, scratch=None) -> EntmaxOpts:
     """Options block. `events`: torch.cuda.Event objects (already recorded once, so that their CUDA handles
     exist) that the call records around its kernel launches (include/entmax_attn.h, per-kernel timing)."""
     o = EntmaxOpts()
@@ -161,6 +166,9 @@ def make_opts(workspace=None, *, scale=0.0, mask_block=0, hist_bins=0, init_mode
     if workspace is not None:
         o.workspace = workspace.data_ptr()
         o.workspace_bytes = workspace.numel() * workspace.element_size()
+    if scratch is not None:
+        o.scratch = scratch.data_ptr()
+        o.scratch_bytes = scratch.numel() * scratch.element_size()
     o.stats = None if stats is None else stats.data_ptr()
     o.tau_hist = None if tau_hist is None else tau_hist.data_ptr()
     o.steps = None if steps is None else steps.data_ptr()
@@ -177,11 +185,22 @@ def entmax_attn_workspace_size(B, H, n, d, dtype_code=ENTMAX_BF16, opts: EntmaxO
                                                  None if opts is None else ctypes.byref(opts)))
 
 
-def alloc_workspace(B, H, n, d, dtype_code=ENTMAX_BF16, device="cuda", opts=None):
+def entmax_attn_saved_size(B, H, n, d, dtype_code=ENTMAX_BF16, opts: EntmaxOpts | None = None) -> int:
+    return int(lib().entmax_attn_saved_size(B, H, n, d, dtype_code, None if opts is None else ctypes.byref(opts)))
+
+
+def entmax_attn_scratch_size(B, H, n, d, dtype_code=ENTMAX_BF16, opts: EntmaxOpts | None = None) -> int:
+    return int(lib().entmax_attn_scratch_size(B, H, n, d, dtype_code, None if opts is None else ctypes.byref(opts)))
+
+
+def alloc_workspace(B, H, n, d, dtype_code=ENTMAX_BF16, device="cuda", opts=None, part="whole"):
+    """Device buffer for the workspace: part "whole" (saved + scratch in one buffer), "saved" or "scratch"."""
     import torch
-    nbytes = entmax_attn_workspace_size(B, H, n, d, dtype_code, opts)
+    size_fn = {"whole": entmax_attn_workspace_size, "saved": entmax_attn_saved_size,
+               "scratch": entmax_attn_scratch_size}[part]
+    nbytes = size_fn(B, H, n, d, dtype_code, opts)
     if nbytes == 0:
-        raise EntmaxError(ENTMAX_ERR_INVALID, "entmax_attn_workspace_size")
+        raise EntmaxError(ENTMAX_ERR_INVALID, size_fn.__name__)
     # torch's caching allocator returns 512-byte aligned blocks
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
@@ -255,14 +274,17 @@ class EntmaxForward:
 
 
 def forward(Q, K, V, alpha, causal=True, *, scale=0.0, mask_block=0, hist_bins=0, init_mode=0,
-            with_stats=False, with_debug=False, stream=None) -> EntmaxForward:
+            with_stats=False, with_debug=False, separate_scratch=False, stream=None) -> EntmaxForward:
+    """Forward with buffers from torch. With separate_scratch, only the workspace's saved part is kept for the
+    backward (the scratch is a transient buffer of this call, and the backward takes its own)."""
     import torch
     B, H, n, d = Q.shape
     dev = Q.device
     mb = mask_block or 64
     code = _dtype_code(Q)
     probe = make_opts(scale=scale, mask_block=mask_block, hist_bins=hist_bins, init_mode=init_mode)
-    ws = alloc_workspace(B, H, n, d, code, dev, probe)
+    ws = alloc_workspace(B, H, n, d, code, dev, probe, part="saved" if separate_scratch else "whole")
+    scratch = alloc_workspace(B, H, n, d, code, dev, probe, part="scratch") if separate_scratch else None
     O = torch.empty_like(Q)
     tau = torch.empty((B, H, n), dtype=torch.float32, device=dev)
     mask = torch.empty(mask_shape(B, H, n, mb), dtype=torch.int32, device=dev)
@@ -270,10 +292,13 @@ def forward(Q, K, V, alpha, causal=True, *, scale=0.0, mask_block=0, hist_bins=0
     tau_hist = torch.empty((B, H, n), dtype=torch.float32, device=dev) if with_debug else None
     steps = torch.empty((B, H, n), dtype=torch.uint8, device=dev) if with_debug else None
     opts = make_opts(ws, scale=scale, mask_block=mask_block, hist_bins=hist_bins, init_mode=init_mode,
-                     stats=stats, tau_hist=tau_hist, steps=steps)
+                     stats=stats, tau_hist=tau_hist, steps=steps, scratch=scratch)
     entmax_attn_fwd(Q, K, V, O, tau, mask, alpha, causal, opts, stream)
+    if separate_scratch:
+        opts = make_opts(ws, scale=scale, mask_block=mask_block, hist_bins=hist_bins, init_mode=init_mode)
     return EntmaxForward(O=O, tau=tau, mask=mask, workspace=ws, opts=opts, stats=stats, tau_hist=tau_hist,
-                         steps=steps, alpha=alpha, causal=causal, keep=(stats, tau_hist, steps))
+                         steps=steps, alpha=alpha, causal=causal, separate=separate_scratch,
+                         keep=(stats, tau_hist, steps))
 
 
 def backward(Q, K, V, fwd: EntmaxForward, dO, stream=None):
@@ -281,7 +306,14 @@ def backward(Q, K, V, fwd: EntmaxForward, dO, stream=None):
     dQ = torch.empty(Q.shape, dtype=torch.float32, device=Q.device)
     dK = torch.empty(K.shape, dtype=torch.float32, device=K.device)
     dV = torch.empty(V.shape, dtype=torch.float32, device=V.device)
-    entmax_attn_bwd(Q, K, V, fwd.O, dO, fwd.tau, fwd.mask, dQ, dK, dV, fwd.alpha, fwd.causal, fwd.opts, stream)
+    opts = fwd.opts
+    if getattr(fwd, "separate", False):
+        B, H, n, d = Q.shape
+        scratch = alloc_workspace(B, H, n, d, _dtype_code(Q), Q.device, fwd.opts, part="scratch")
+        opts = EntmaxOpts.from_buffer_copy(fwd.opts)
+        opts.scratch = scratch.data_ptr()
+        opts.scratch_bytes = scratch.numel()
+    entmax_attn_bwd(Q, K, V, fwd.O, dO, fwd.tau, fwd.mask, dQ, dK, dV, fwd.alpha, fwd.causal, opts, stream)
     return dQ, dK, dV
 
 

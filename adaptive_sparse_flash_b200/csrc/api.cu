@@ -118,23 +118,30 @@ entmax_status check_dims(int B, int H, int n, int d, entmax_dtype dt, const entm
     return ENTMAX_OK;
 }
 
-// Workspace: U V (fp32 [BH][n][d]) and sum u ([BH][n]) from the forward; delta and the row statistic
-// padded to whole 64-row blocks ([BH][ceil(n/64)*64]) for the backward; the transposed mask.
+// Workspace, in two parts.
+//   saved   - what the backward needs from the forward: U V (fp32 [BH][n][d]), sum u ([BH][n]) and the
+//             transposed mask;
+//   scratch - per call: delta and the row statistic padded to whole 64-row blocks ([BH][ceil(n/64)*64]) for
+//             the backward, the range words, and the fp16 operand copies of Q, K, V, dO (f16.cu).
+// With one buffer (opts->scratch NULL) the scratch part follows the saved part, and a backward reuses the
+// fp16 copies its forward left there; with a separate scratch buffer the backward makes its own copies.
 struct Workspace {
     float* obar;
     float* sum_u;
+    uint32_t* maskT;
     float* delta_pad;
     float* stat_pad;
-    uint32_t* maskT;
-    uint32_t* maxbits;  // [8]: max |x| of Q, K, V (forward), dO (backward), as float bits
+    uint32_t* maxbits;  // [8]: max |x| of Q, K, V, dO, as float bits
     void* Qh;           // fp16 copies [BH][n][d] (f16.cu)
     void* Kh;
     void* Vh;
     void* dOh;
-    size_t bytes;
+    size_t saved_bytes;
+    size_t scratch_bytes;
+    bool separate;      // scratch in its own buffer
 };
 
-Workspace layout(const Dims& D, void* base) {
+Workspace layout(const Dims& D, void* base, void* scratch) {
     const size_t rows = (size_t)D.B * D.H * D.n;
     const size_t rows_pad = (size_t)D.B * D.H * (size_t)((D.n + 63) / 64) * 64;
     Workspace w;
@@ -144,28 +151,37 @@ Workspace layout(const Dims& D, void* base) {
     off = align256(off + rows * D.d * sizeof(float));
     w.sum_u = reinterpret_cast<float*>(p + off);
     off = align256(off + rows * sizeof(float));
-    w.delta_pad = reinterpret_cast<float*>(p + off);
-    off = align256(off + rows_pad * sizeof(float));
-    w.stat_pad = reinterpret_cast<float*>(p + off);
-    off = align256(off + rows_pad * sizeof(float));
     w.maskT = reinterpret_cast<uint32_t*>(p + off);
     off = align256(off + (size_t)D.B * D.H * D.nkb * D.nwq * sizeof(uint32_t));
-    w.maxbits = reinterpret_cast<uint32_t*>(p + off);
-    off = align256(off + 8 * sizeof(uint32_t));
+    w.saved_bytes = off;
+    w.separate = scratch != nullptr;
+    char* q = scratch ? static_cast<char*>(scratch) : p + off;
+    size_t so = 0;
+    w.delta_pad = reinterpret_cast<float*>(q + so);
+    so = align256(so + rows_pad * sizeof(float));
+    w.stat_pad = reinterpret_cast<float*>(q + so);
+    so = align256(so + rows_pad * sizeof(float));
+    w.maxbits = reinterpret_cast<uint32_t*>(q + so);
+    so = align256(so + 8 * sizeof(uint32_t));
     void** h16[4] = {&w.Qh, &w.Kh, &w.Vh, &w.dOh};
     for (int i = 0; i < 4; ++i) {
-        *h16[i] = p + off;
-        off = align256(off + rows * D.d * 2);
+        *h16[i] = q + so;
+        so = align256(so + rows * D.d * 2);
     }
-    w.bytes = off;
+    w.scratch_bytes = so;
     return w;
 }
 
 entmax_status check_workspace(const Dims& D, const entmax_opts* o, Workspace* w) {
     if (!o || !o->workspace) return ENTMAX_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(o->workspace) & 255u) != 0) return ENTMAX_ERR_ALIGN;
-    *w = layout(D, o->workspace);
-    if (o->workspace_bytes < w->bytes) return ENTMAX_ERR_WORKSPACE;
+    if (o->scratch && (reinterpret_cast<uintptr_t>(o->scratch) & 255u) != 0) return ENTMAX_ERR_ALIGN;
+    *w = layout(D, o->workspace, o->scratch);
+    if (o->scratch) {
+        if (o->workspace_bytes < w->saved_bytes || o->scratch_bytes < w->scratch_bytes) return ENTMAX_ERR_WORKSPACE;
+    } else if (o->workspace_bytes < w->saved_bytes + w->scratch_bytes) {
+        return ENTMAX_ERR_WORKSPACE;
+    }
     return ENTMAX_OK;
 }
 
@@ -218,7 +234,20 @@ EATTN_API const char* entmax_status_str(entmax_status s) {
 EATTN_API size_t entmax_attn_workspace_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts) {
     Dims D;
     if (check_dims(B, H, n, d, dt, opts, &D) != ENTMAX_OK) return 0;
-    return layout(D, nullptr).bytes;
+    const Workspace w = layout(D, nullptr, nullptr);
+    return w.saved_bytes + w.scratch_bytes;
+}
+
+EATTN_API size_t entmax_attn_saved_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts) {
+    Dims D;
+    if (check_dims(B, H, n, d, dt, opts, &D) != ENTMAX_OK) return 0;
+    return layout(D, nullptr, nullptr).saved_bytes;
+}
+
+EATTN_API size_t entmax_attn_scratch_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts) {
+    Dims D;
+    if (check_dims(B, H, n, d, dt, opts, &D) != ENTMAX_OK) return 0;
+    return layout(D, nullptr, nullptr).scratch_bytes;
 }
 
 EATTN_API entmax_status entmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* tau,
@@ -354,14 +383,22 @@ entmax_status bwd_common(const void* Q, const void* K, const void* V, const void
         return from_cuda(e);
     }
     if (!softmax && use_f16_path(d, alpha, D.nw, D.bins)) {
-        // fp16 path: the forward left fp16 copies of Q, K, V and their range exponents in the workspace
+        // fp16 path: with one workspace buffer the forward left fp16 copies of Q, K, V and their range
+        // exponents in it and only dO is converted here; with a separate scratch buffer all four are
         F16Job job;
         memset(&job, 0, sizeof(job));
-        job.src[0] = dO;
-        job.dst[0] = ws.dOh;
-        job.maxbits = ws.maxbits + 3;
+        if (ws.separate) {
+            job.src[0] = Q; job.src[1] = K; job.src[2] = V; job.src[3] = dO;
+            job.dst[0] = ws.Qh; job.dst[1] = ws.Kh; job.dst[2] = ws.Vh; job.dst[3] = ws.dOh;
+            job.maxbits = ws.maxbits;
+            job.count = 4;
+        } else {
+            job.src[0] = dO;
+            job.dst[0] = ws.dOh;
+            job.maxbits = ws.maxbits + 3;
+            job.count = 1;
+        }
         job.n16 = (size_t)B * H * n * d / 8;
-        job.count = 1;
         a.Qh = ws.Qh; a.Kh = ws.Kh; a.Vh = ws.Vh; a.dOh = ws.dOh; a.maxbits = ws.maxbits;
         cudaError_t e = launch_to_f16(job, num_sms(), s);
         if (e == cudaSuccess) e = launch_bwd_h(a, ws.delta_pad, ws.stat_pad, s);
@@ -468,6 +505,8 @@ EATTN_API entmax_status entmax_attn_fwd_noalloc(const void* Q, const void* K, co
     entmax_opts o;
     memset(&o, 0, sizeof(o));
     if (opts) o = *opts;
+    o.scratch = nullptr;
+    o.scratch_bytes = 0;
     const size_t need = entmax_attn_workspace_size(B, H, n, d, dt, &o);
     if (need == 0) {
         // let the regular checks name the problem (invalid or unsupported sizes)
@@ -482,6 +521,8 @@ EATTN_API entmax_status entmax_attn_fwd_noalloc(const void* Q, const void* K, co
     if (!scratch) return ENTMAX_ERR_CUDA;
     o.workspace = scratch;
     o.workspace_bytes = kStaticScratchBytes;
+    o.scratch = nullptr;
+    o.scratch_bytes = 0;
     return entmax_attn_fwd(Q, K, V, O, tau, block_mask, B, H, n, d, alpha, causal, dt, &o, stream);
 }
 

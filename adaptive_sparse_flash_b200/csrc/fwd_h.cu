@@ -69,10 +69,13 @@ constexpr uint32_t offHist = offK + NKS * kKBytes;
 
 // Shared-memory plan for up to NB histogram bins (256, or 512): the histogram u16 [NB][128] (the V ring of
 // P V sweeps reuses it), then the candidate stash fp32 [2][kHalf][128]. At 512 bins the histogram takes
-// 128 KB and the stash shrinks to 28 entries per row and warpgroup, so that the CTA still fits.
+// 128 KB and the stash shrinks to 32 entries per row and warpgroup, so that the CTA still fits. The
+// histogram sweep of an overflowed row stages a whole 64-key block in that row's stash slots, from the
+// start of warpgroup 0's half: the two halves together must hold 64 entries.
 template <int NB>
 struct HCfg {
-    static constexpr int kHalf = NB == 512 ? 28 : 88;  // stash entries per row and warpgroup
+    static constexpr int kHalf = NB == 512 ? 32 : 88;  // stash entries per row and warpgroup
+    static_assert(2 * kHalf >= BN, "the histogram sweep stages a 64-key block in a row's stash slots");
     static constexpr uint32_t kHistBytes = (uint32_t)NB * BM * 2u;
     static constexpr uint32_t kStashBytes = 2u * kHalf * BM * 4u;
     static constexpr uint32_t offStash = offHist + kHistBytes;
@@ -628,14 +631,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const bool keep = amax > thr_f;
                         if (__any_sync(0xffffffffu, mine && keep)) {
                             if (mine && keep) {
-                                // stage the block in the row's stash slots (no longer needed) and bin it
-                                // with a rolled loop
+                                // stage the block in the row's stash slots (no longer needed; this is
+                                // warpgroup 0, so the slots from the start of the stash, both halves: 2 kHalf
+                                // >= 64) and bin it with a rolled loop
                                 uint32_t gflag = 0u;
 #pragma unroll
                                 for (int q = 0; q < 8; ++q) gflag |= (gm[q] > thr_f ? 1u : 0u) << q;
 #pragma unroll
-                                for (int c = 0; c < BN; ++c) st_mine[c * BM + r] = vbuf[c];
-                                hist_bin_block(h, st_mine + r, gflag, sp, hist, r);
+                                for (int c = 0; c < BN; ++c) stash[c * BM + r] = vbuf[c];
+                                hist_bin_block(h, stash + r, gflag, sp, hist, r);
                             }
                         }
                         const uint32_t ball = __ballot_sync(0xffffffffu, keep);
@@ -752,72 +756,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float amax = group_max();
                     const bool keep = sp.cz * amax > lo0;
                     const bool nz = fmaf(amax, sp.cz, -t) > 0.f;
-                    // two branch-free passes over the block, P then U, through one 32-word array; the solver
-                    // sums ride on the P pass, in warps that hold a row whose tau still needs the check
-                    uint32_t w32[32];
-                    auto p_pass = [&](auto with_sums) {
+                    // one branch-free pass over the block, 32 keys at a time: p and u of each key, packed as
+                    // fp16 pairs into the columns of the S tile just read (this warpgroup's own buffer), P in
+                    // the first 32 columns and U in the next 32. The solver sums ride along in warps that hold
+                    // a row whose tau still needs the check.
+                    const uint32_t tp = lane_base + colS;
+                    auto pu_pass = [&](auto with_sums) {
                         constexpr bool SUMS = decltype(with_sums)::value;
 #pragma unroll
-                        for (int c = 0; c < BN; c += 2) {
-                            float p2[2];
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t wp[16], wu[16];
 #pragma unroll
-                            for (int h2 = 0; h2 < 2; ++h2) {
-                                const float x = fmaf(vbuf[c + h2], sp.cz, -t);
-                                float pp, uu;
-                                if constexpr (KIND == kAlpha15) {
-                                    uu = fmaxf(x, 0.f);
-                                    pp = uu * uu;
-                                    if constexpr (SUMS) F2 += x > 0.f ? 1.f : 0.f;
-                                } else if constexpr (KIND == kAlpha2) {
-                                    pp = fmaxf(x, 0.f);
-                                    uu = x > 0.f ? 1.f : 0.f;
-                                } else {
-                                    const bool pos = x > 0.f;
-                                    const float xs = pos ? x : 1.f;
-                                    const float u1 = exp2f((sp.k - 1.f) * __log2f(xs));
-                                    uu = pos ? u1 : 0.f;
-                                    pp = uu * xs;
-                                    if constexpr (SUMS) F2 += pos ? __fdividef(u1, xs) : 0.f;
+                            for (int c = 0; c < 32; c += 2) {
+                                float p2[2], u2[2];
+#pragma unroll
+                                for (int h2 = 0; h2 < 2; ++h2) {
+                                    const float x = fmaf(vbuf[32 * h + c + h2], sp.cz, -t);
+                                    float pp, uu;
+                                    if constexpr (KIND == kAlpha15) {
+                                        uu = fmaxf(x, 0.f);
+                                        pp = uu * uu;
+                                        if constexpr (SUMS) F2 += x > 0.f ? 1.f : 0.f;
+                                    } else if constexpr (KIND == kAlpha2) {
+                                        pp = fmaxf(x, 0.f);
+                                        uu = x > 0.f ? 1.f : 0.f;
+                                    } else {
+                                        const bool pos = x > 0.f;
+                                        const float xs = pos ? x : 1.f;
+                                        const float u1 = exp2f((sp.k - 1.f) * __log2f(xs));
+                                        uu = pos ? u1 : 0.f;
+                                        pp = uu * xs;
+                                        if constexpr (SUMS) F2 += pos ? __fdividef(u1, xs) : 0.f;
+                                    }
+                                    if constexpr (SUMS) {
+                                        Sp += pp;
+                                        Sq += uu;
+                                        Sn += x > 0.f ? 1u : 0u;
+                                    }
+                                    p2[h2] = pp;
+                                    u2[h2] = uu;
                                 }
-                                if constexpr (SUMS) {
-                                    Sp += pp;
-                                    Sq += uu;
-                                    Sn += x > 0.f ? 1u : 0u;
-                                }
-                                p2[h2] = pp;
+                                wp[c / 2] = pack_half2(p2[0], p2[1]);
+                                wu[c / 2] = pack_half2(u2[0], u2[1]);
                             }
-                            w32[c / 2] = pack_half2(p2[0], p2[1]);
+                            tmem_st16(tp + 16 * h, wp);
+                            tmem_st16(tp + 32 + 16 * h, wu);
                         }
                     };
-                    if (need_sums) p_pass(std::true_type{});
-                    else p_pass(std::false_type{});
-                    // P and U go into the columns of the S tile just read (this warpgroup's own buffer)
-                    const uint32_t tp = lane_base + colS;
-                    tmem_st32(tp, w32);
-                    // U next to P, one fp16 term, in two halves of 32 keys
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t wu[16];
-#pragma unroll
-                        for (int c = 0; c < 32; c += 2) {
-                            float u2[2];
-#pragma unroll
-                            for (int h2 = 0; h2 < 2; ++h2) {
-                                const float x = fmaf(vbuf[32 * h + c + h2], sp.cz, -t);
-                                if constexpr (KIND == kAlpha15) {
-                                    u2[h2] = fmaxf(x, 0.f);
-                                } else if constexpr (KIND == kAlpha2) {
-                                    u2[h2] = x > 0.f ? 1.f : 0.f;
-                                } else {
-                                    const bool pos = x > 0.f;
-                                    const float xs = pos ? x : 1.f;
-                                    u2[h2] = pos ? exp2f((sp.k - 1.f) * __log2f(xs)) : 0.f;
-                                }
-                            }
-                            wu[c / 2] = pack_half2(u2[0], u2[1]);
-                        }
-                        tmem_st16(tp + 32 + 16 * h, wu);
-                    }
+                    if (need_sums) pu_pass(std::true_type{});
+                    else pu_pass(std::false_type{});
                     tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();

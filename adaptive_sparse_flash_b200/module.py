@@ -23,8 +23,10 @@ __all__ = ["EntmaxAttnFunction", "entmax_attention", "EntmaxMultiheadAttention"]
 class EntmaxAttnFunction(torch.autograd.Function):
     """O = alpha-entmax(scale Q K^T) V for bf16 [B, H, n, d] tensors on a CUDA device (d in {64, 128}).
 
-    The forward keeps the library's workspace (which holds what its backward reads), tau and the block
-    mask for the backward. Gradients come back in the inputs' dtype (the library computes them in fp32).
+    Besides q, k, v and O, the forward keeps tau, the block mask and the saved part of the library's
+    workspace (U V in fp32, sum u, the transposed mask) for the backward; the fp16 operand copies live in a
+    per-call scratch buffer, so they are not activation memory. Gradients come back in the inputs' dtype
+    (the library computes them in fp32).
     """
 
     @staticmethod
@@ -33,7 +35,7 @@ class EntmaxAttnFunction(torch.autograd.Function):
             if not t.is_cuda or t.dtype != torch.bfloat16:
                 raise TypeError("entmax attention takes bf16 CUDA tensors")
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        f = _b.forward(q, k, v, alpha, causal, scale=scale, hist_bins=hist_bins)
+        f = _b.forward(q, k, v, alpha, causal, scale=scale, hist_bins=hist_bins, separate_scratch=True)
         ctx.save_for_backward(q, k, v, f.O, f.tau, f.mask, f.workspace)
         ctx.alpha, ctx.causal, ctx.scale, ctx.hist_bins = alpha, causal, scale, hist_bins
         return f.O
@@ -42,7 +44,10 @@ class EntmaxAttnFunction(torch.autograd.Function):
     def backward(ctx, dO):
         q, k, v, O, tau, mask, ws = ctx.saved_tensors
         dO = dO.to(torch.bfloat16).contiguous()
-        opts = _b.make_opts(ws, scale=ctx.scale, hist_bins=ctx.hist_bins)
+        Bsz, H, n, d = q.shape
+        probe = _b.make_opts(scale=ctx.scale, hist_bins=ctx.hist_bins)
+        scratch = _b.alloc_workspace(Bsz, H, n, d, _b.ENTMAX_BF16, q.device, probe, part="scratch")
+        opts = _b.make_opts(ws, scale=ctx.scale, hist_bins=ctx.hist_bins, scratch=scratch)
         dQ, dK, dV = (torch.empty(x.shape, dtype=torch.float32, device=x.device) for x in (q, k, v))
         _b.entmax_attn_bwd(q, k, v, O, dO, tau, mask, dQ, dK, dV, ctx.alpha, ctx.causal, opts)
         return dQ.to(q.dtype), dK.to(k.dtype), dV.to(v.dtype), None, None, None, None

@@ -126,7 +126,9 @@ def bins_report(out=sys.stdout):
 
 def memory_report(out=sys.stdout):
     """Device bytes that stay allocated between the forward and the backward (the activation memory of the
-    attention), measured with torch's allocator around each call, and the peak during the backward."""
+    attention), measured with torch's allocator around each call, and the peak during the backward.
+    Three paths: entmax with one workspace buffer (the fp16 operand copies are kept for the backward),
+    entmax with a separate per-call scratch (only the saved part is kept), and the dense softmax baseline."""
     import torch
 
     from . import binding as b
@@ -139,11 +141,11 @@ def memory_report(out=sys.stdout):
         t = _to_dev(arr)
         Q, K, V, dO = t["Q"], t["K"], t["V"], t["dO"]
         alpha = alphas[0]
-        for path in ("entmax", "softmax"):
+        for path in ("entmax, one buffer", "entmax, separate scratch", "softmax"):
             torch.cuda.synchronize()
             base = torch.cuda.memory_allocated()
-            if path == "entmax":
-                f = b.forward(Q, K, V, alpha, True)
+            if path.startswith("entmax"):
+                f = b.forward(Q, K, V, alpha, True, separate_scratch=path.endswith("scratch"))
                 kept = (f.O, f.tau, f.mask, f.workspace)
                 ws_bytes = f.workspace.numel()
             else:
@@ -153,7 +155,7 @@ def memory_report(out=sys.stdout):
             torch.cuda.synchronize()
             after_fwd = torch.cuda.memory_allocated() - base
             torch.cuda.reset_peak_memory_stats()
-            if path == "entmax":
+            if path.startswith("entmax"):
                 g = b.backward(Q, K, V, f, dO)
             else:
                 g = b.softmax_backward(Q, K, V, O, lse, dO, True)
@@ -162,7 +164,7 @@ def memory_report(out=sys.stdout):
             print(f"| {name} B={B} H={H} n={n} d={d} | {path} | {after_fwd / mib:.1f} | {ws_bytes / mib:.1f} | "
                   f"{peak / mib:.1f} |", file=out, flush=True)
             del kept, g
-            if path == "entmax":
+            if path.startswith("entmax"):
                 del f
             else:
                 del O, lse

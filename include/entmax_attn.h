@@ -85,7 +85,21 @@ typedef struct {
     uint8_t* steps;         /* optional device [B,H,n]: solver steps taken by each row             */
     void* const* events;    /* optional cudaEvent_t handles (as void*) for per-kernel timing, or NULL */
     int num_events;         /* length of `events` (0 when NULL); see "Per-kernel timing" below       */
+    void* scratch;          /* optional per-call scratch (>= entmax_attn_scratch_size() bytes, 256-aligned);
+                               NULL: the scratch lies inside the workspace (see "Workspace" below)    */
+    size_t scratch_bytes;
 } entmax_opts;
+
+/* Workspace. The library's device scratch has two parts:
+ *   saved   - written by the forward and read by its backward: U V (fp32 [B,H,n,d]), sum u (fp32 [B,H,n])
+ *             and the transposed block mask; entmax_attn_saved_size() bytes;
+ *   scratch - used within one call: the fp16 operand copies of Q, K, V, dO, the padded per-row delta and
+ *             row statistic, range words; entmax_attn_scratch_size() bytes.
+ * With opts->scratch NULL, opts->workspace holds both (entmax_attn_workspace_size() bytes, the sum) and a
+ * backward reuses the fp16 copies of Q, K, V that its forward left there. With opts->scratch set,
+ * opts->workspace needs only the saved part: only that must be kept from the forward to the backward (the
+ * activation memory of the attention is then O, tau, the mask and the saved part), and the backward
+ * makes its own fp16 copies in whatever scratch it is given. */
 
 /* Per-kernel timing. When opts->events is set, a call records events[i] on `stream` right before its i-th
  * kernel launch and one more event after its last launch (events past num_events are not recorded; a NULL
@@ -102,9 +116,15 @@ typedef struct {
  * The events are recorded by the host thread that makes the call, as part of it; opts->events must stay
  * valid for the duration of the call only. */
 
-/* Bytes of workspace that entmax_attn_fwd/bwd (or softmax_attn_fwd/bwd) need for these sizes.
- * Returns 0 for invalid sizes. opts may be NULL (defaults). */
+/* Bytes of workspace that entmax_attn_fwd/bwd (or softmax_attn_fwd/bwd) need for these sizes, saved and
+ * scratch parts together (a single buffer, opts->scratch NULL). Returns 0 for invalid sizes. opts may be
+ * NULL (defaults). */
 size_t entmax_attn_workspace_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts);
+
+/* Bytes of the saved part alone (opts->workspace when opts->scratch is set), and of the scratch part
+ * (opts->scratch). 0 for invalid sizes. */
+size_t entmax_attn_saved_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts);
+size_t entmax_attn_scratch_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts);
 
 /* Forward. Q, K, V: [B,H,n,d] inputs. O: [B,H,n,d] output (same dtype). tau: float32 [B,H,n]
  * output, the normaliser in z units. block_mask: uint32 output as described above. alpha > 1.
@@ -143,7 +163,7 @@ entmax_status softmax_attn_bwd(const void* Q, const void* K, const void* V, cons
  * callers that cannot allocate device memory, e.g. code running inside a framework that owns the whole
  * device pool, or paths that must not call cudaMalloc, which may synchronise and is not allowed during
  * stream capture). Same arguments, outputs and checks as entmax_attn_fwd; opts may be NULL and any
- * opts->workspace is ignored. The scratch lives in a 32 MiB (33554432-byte) device array inside the
+ * opts->workspace and opts->scratch are ignored. The scratch lives in a 32 MiB (33554432-byte) device array inside the
  * library, which every GPU that loads the library holds until exit; calls whose workspace
  * (entmax_attn_workspace_size) would be larger return ENTMAX_ERR_WORKSPACE. The first call on
  * each device looks up the array's device address (cudaGetSymbolAddress), so make that first call
@@ -168,7 +188,8 @@ entmax_status entmax_attn_selftest_timeout(int limit_us, void* stream);
 /* Human-readable name of a status code (static string). */
 const char* entmax_status_str(entmax_status s);
 
-/* Library ABI version: 2 (entmax_opts gained `events` and `num_events`). */
+/* Library ABI version: 2 (entmax_opts gained `events`, `num_events`, `scratch`, `scratch_bytes`; entmax_stats
+ * gained `support`; entmax_attn_saved_size and entmax_attn_scratch_size were added). */
 int entmax_attn_version(void);
 
 #ifdef __cplusplus

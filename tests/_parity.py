@@ -53,10 +53,10 @@ def check_mask(mask_gpu_words, bits_ref, bmax_ref, where=""):
 
 
 def grad_sensitivity(q, k, v, do, alpha, causal, scale=None):
-    """Bounds on the gradient error that float32 scores alone can cause, for one head (float64).
+    """Bounds on the output and gradient error that float32 scores alone can cause, for one head (float64).
 
-    Returns (dQ per query row, dK per key column, dV per key column) bounds of the max abs change of each
-    row / column when every score z_ij moves by up to
+    Returns (dQ per query row, dK per key column, dV per key column, O per query row) bounds of the max abs
+    change of each row / column when every score z_ij moves by up to
 
         eps_ij = 2^-21 |z|_ij  +  1e-5 / (k sum_j u_ij)  +  4 ulp_f32(tau_i)
 
@@ -68,8 +68,8 @@ def grad_sensitivity(q, k, v, do, alpha, causal, scale=None):
         over the entries that are or may become support, and by M_i R_i / (sum u - M_i) while the unstable
         u mass M_i = sum_j du_ij is below half of sum u;
       * dS_ij = u_ij (g_ij - delta_i) then moves by du_ij |g_ij - delta_i| + (u_ij + du_ij) d delta_i, and
-        dQ_i = scale sum_j dS_ij k_j, dK_j = scale sum_i dS_ij q_i, dV_j = sum_i p_ij dO_i by the sums of
-        those changes times the max-norm of k_j, q_i, dO_i.
+        dQ_i = scale sum_j dS_ij k_j, dK_j = scale sum_i dS_ij q_i, dV_j = sum_i p_ij dO_i, O_i = sum_j p_ij v_j
+        by the sums of those changes times the max-norm of k_j, q_i, dO_i, v_j.
     For alpha < 2 u is continuous in x and the bounds are tiny; for alpha > 2 u = x^(k-1) is unbounded as
     x -> 0+ (alpha = 3: u = x^-1/2), so a row with a support entry within rounding of tau has gradients
     that no float32 computation of the scores determines.
@@ -108,7 +108,8 @@ def grad_sensitivity(q, k, v, do, alpha, causal, scale=None):
     kinf = np.abs(k64).max(1)
     qinf = np.abs(q64).max(1)
     doinf = np.abs(np.asarray(do, np.float64)).max(1)
-    return scale * dds @ kinf, scale * qinf @ dds, doinf @ dp
+    vinf = np.abs(np.asarray(v, np.float64)).max(1)
+    return scale * dds @ kinf, scale * qinf @ dds, doinf @ dp, dp @ vinf
 
 
 def check_grads_bounded(gpu, ref, sens, where, max_abs=BF16_MAX_ABS, mean_abs=BF16_MEAN_ABS, cap=None):
