@@ -239,7 +239,6 @@ __device__ __forceinline__ void stash_sums(const Stash& st, const float* stash, 
 template <int KIND>
 __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, const uint16_t* hist, int r, const float* T) {
     const int B = sp.bins;
-    const float Bm1 = (float)(B - 1);
     auto cnt = [&](int j) -> uint32_t {
         const int sl = (h.top - j) & (B - 1);
         return ((h.live[sl >> 5] >> (sl & 31)) & 1u) ? (uint32_t)hist[sl * kTileRows + r] : 0u;

@@ -54,7 +54,7 @@ constexpr int BN = 64;
 constexpr int D = 64;
 constexpr int kThreads = 352;
 constexpr int kCompute = 256;
-constexpr int NKS = 4;
+constexpr int NKS_MAX = 8;  // K ring stages, at most
 constexpr int NVS = 8;
 constexpr int NSB = 3;  // S buffers per compute warpgroup
 
@@ -65,7 +65,6 @@ constexpr uint32_t kKBytes = BN * D * 2;                 // 8 KB per K or V bloc
 constexpr uint32_t kQBytes = BM * D * 2;                 // 16 KB
 constexpr uint32_t offQ = 0;
 constexpr uint32_t offK = offQ + kQBytes;
-constexpr uint32_t offHist = offK + NKS * kKBytes;
 
 // Shared-memory plan for up to NB histogram bins (256, or 512): the histogram u16 [NB][128] (the V ring of
 // P V sweeps reuses it), then the candidate stash fp32 [2][kHalf][128]. At 512 bins the histogram takes
@@ -74,7 +73,10 @@ constexpr uint32_t offHist = offK + NKS * kKBytes;
 // start of warpgroup 0's half: the two halves together must hold 64 entries.
 template <int NB>
 struct HCfg {
+    static constexpr int kNKS = 4;                     // K ring stages
     static constexpr int kHalf = NB == 512 ? 32 : 88;  // stash entries per row and warpgroup
+    static constexpr uint32_t offHist = offK + kNKS * kKBytes;
+    static_assert(kNKS <= NKS_MAX, "K ring barriers");
     static_assert(2 * kHalf >= BN, "the histogram sweep stages a 64-key block in a row's stash slots");
     static constexpr uint32_t kHistBytes = (uint32_t)NB * BM * 2u;
     static constexpr uint32_t kStashBytes = 2u * kHalf * BM * 4u;
@@ -102,7 +104,7 @@ enum : int {
 
 struct Small {
     uint64_t q_full;
-    uint64_t k_full[NKS], k_empty[NKS];
+    uint64_t k_full[NKS_MAX], k_empty[NKS_MAX];
     uint64_t v_full[NVS], v_empty[NVS];
     uint64_t s_full[2][NSB], s_empty[2][NSB];  // [warpgroup][buffer]
     uint64_t pv_free[2][NSB];                  // P V products that read a buffer's P and U have completed
@@ -215,6 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fwd_h_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const FwdArgs a) {
     using HC = HCfg<NB>;
+    constexpr int NKS = HC::kNKS;
+    constexpr uint32_t offHist = HC::offHist;
     constexpr int kHalf = HC::kHalf;
     constexpr uint32_t offStash = HC::offStash;
     constexpr uint32_t offV = HC::offV;

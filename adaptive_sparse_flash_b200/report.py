@@ -5,6 +5,8 @@
     python -m adaptive_sparse_flash_b200.report bins     # histogram size B: iterations, shared memory, time
     python -m adaptive_sparse_flash_b200.report memory   # bytes kept from forward to backward, entmax and
                                                          # the in-library dense softmax baseline
+    python -m adaptive_sparse_flash_b200.report timing   # per configuration: forward / backward ms, effective
+                                                         # TFLOP/s, the dense baseline on the same inputs
 
 The solver report covers the pages' iteration claims: one or two solver steps after the histogram start,
 against five to ten without it (euno.news summary, "方法论" item 3; gist.science (de), section 2,
@@ -171,13 +173,92 @@ def memory_report(out=sys.stdout):
         del t, Q, K, V, dO
 
 
+def _peak_burst():
+    import json
+    import os
+    p = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            return float(json.load(fh).get("bf16_tflops", 1590.0)), "measured"
+    return 1590.0, "fallback"
+
+
+def timing_report(out=sys.stdout):
+    """Per configuration: entmax forward and backward ms (median of 5 CUDA-event timed calls, L2 flushed
+    before each), effective TFLOP/s (dense Q K^T over the causal entries plus the P V and, for fwd + bwd
+    configurations, the five backward products of each nonzero 64 x 64 block), its fraction of the bf16
+    burst peak, and the dense softmax baseline of the library on the same inputs."""
+    import numpy as np
+    import torch
+
+    from . import binding as b
+    peak, src = _peak_burst()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def timed(fn, reps=5):
+        fn()
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return sorted(ts)[len(ts) // 2]
+
+    print(f"| workload | alpha | pass | entmax fwd ms | entmax bwd ms | effective TFLOP/s | frac of bf16 burst "
+          f"({peak:g}, {src}) | dense fwd (+bwd) ms | block sparsity |", file=out)
+    print("|---|---|---|---|---|---|---|---|---|", file=out)
+    for name, kind, B, H, n, d, alphas, psets in CONFIGS:
+        for params in psets:
+            arr = _gen(kind, B, H, n, d, params)
+            t = _to_dev(arr)
+            Q, K, V, dO = t["Q"], t["K"], t["V"], t["dO"]
+            fwd_only = name == "cfg2"
+            ws = b.alloc_workspace(B, H, n, d)
+            opts = b.make_opts(ws)
+            O = torch.empty_like(Q)
+            tau = torch.empty((B, H, n), dtype=torch.float32, device="cuda")
+            mask = torch.empty(b.mask_shape(B, H, n), dtype=torch.int32, device="cuda")
+            gq, gk, gv = (torch.empty(Q.shape, dtype=torch.float32, device="cuda") for _ in range(3))
+            lse = torch.empty((B, H, n), dtype=torch.float32, device="cuda")
+            for alpha in alphas:
+                fwd = lambda: b.entmax_attn_fwd(Q, K, V, O, tau, mask, alpha, True, opts)  # noqa: E731
+                fms = timed(fwd)
+                fwd()
+                torch.cuda.synchronize()
+                nnz = int(np.unpackbits(mask.cpu().numpy().view(np.uint8), bitorder="little").sum())
+                nqb = (n + 63) // 64
+                qk = 2.0 * d * n * (n + 1) / 2 * B * H
+                blk = 2.0 * d * 64 * 64 * nnz
+                if fwd_only:
+                    bms = float("nan")
+                    flops, ms = qk + blk, fms
+                    dense = timed(lambda: b.softmax_attn_fwd(Q, K, V, O, lse, True, opts))
+                else:
+                    bwd = lambda: b.entmax_attn_bwd(Q, K, V, O, dO, tau, mask, gq, gk, gv, alpha, True, opts)  # noqa
+                    bms = timed(lambda: (fwd(), bwd())) - fms
+                    flops, ms = qk + 6 * blk, fms + bms
+                    dense = timed(lambda: (b.softmax_attn_fwd(Q, K, V, O, lse, True, opts),
+                                           b.softmax_attn_bwd(Q, K, V, O, dO, lse, gq, gk, gv, True, opts)))
+                tf = flops / (ms * 1e-3) / 1e12
+                label = f"{name} {' '.join(f'{k}={v:g}' for k, v in params.items())} B={B} H={H} n={n} d={d}"
+                print(f"| {label} | {alpha:g} | {'fwd' if fwd_only else 'fwd+bwd'} | {fms:.3f} | "
+                      f"{'-' if fwd_only else f'{bms:.3f}'} | {tf:.1f} | {tf / peak:.3f} | {dense:.3f} | "
+                      f"{1 - nnz / (B * H * nqb * (nqb + 1) // 2):.3f} |", file=out, flush=True)
+            del t, Q, K, V, dO, ws
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
-    ap.add_argument("what", choices=["solver", "bins", "memory"])
+    ap.add_argument("what", choices=["solver", "bins", "memory", "timing"])
     args = ap.parse_args(argv)
     from . import build
     build.build()
-    {"solver": solver_report, "bins": bins_report, "memory": memory_report}[args.what]()
+    {"solver": solver_report, "bins": bins_report, "memory": memory_report, "timing": timing_report}[args.what]()
 
 
 if __name__ == "__main__":
