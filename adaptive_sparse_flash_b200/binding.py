@@ -81,6 +81,7 @@ class EntmaxOpts(ctypes.Structure):
         ("num_events", ctypes.c_int),
         ("scratch", ctypes.c_void_p),
         ("scratch_bytes", ctypes.c_size_t),
+        ("alpha", ctypes.c_float),
     ]
 
 
@@ -155,7 +156,7 @@ def _dtype_code(t) -> int:
 
 
 def make_opts(workspace=None, *, scale=0.0, mask_block=0, hist_bins=0, init_mode=0,
-              stats=None, tau_hist=None, steps=None, events=None, scratch=None) -> EntmaxOpts:
+              stats=None, tau_hist=None, steps=None, events=None, scratch=None, alpha=0.0) -> EntmaxOpts:
     """Options block. `events`: torch.cuda.Event objects (already recorded once, so that their CUDA handles
     exist) that the call records around its kernel launches (include/entmax_attn.h, per-kernel timing)."""
     o = EntmaxOpts()
@@ -163,6 +164,7 @@ def make_opts(workspace=None, *, scale=0.0, mask_block=0, hist_bins=0, init_mode
     o.mask_block = int(mask_block)
     o.hist_bins = int(hist_bins)
     o.init_mode = int(init_mode)
+    o.alpha = float(alpha)
     if workspace is not None:
         o.workspace = workspace.data_ptr()
         o.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -282,7 +284,7 @@ def forward(Q, K, V, alpha, causal=True, *, scale=0.0, mask_block=0, hist_bins=0
     dev = Q.device
     mb = mask_block or 64
     code = _dtype_code(Q)
-    probe = make_opts(scale=scale, mask_block=mask_block, hist_bins=hist_bins, init_mode=init_mode)
+    probe = make_opts(scale=scale, mask_block=mask_block, hist_bins=hist_bins, init_mode=init_mode, alpha=alpha)
     ws = alloc_workspace(B, H, n, d, code, dev, probe, part="saved" if separate_scratch else "whole")
     scratch = alloc_workspace(B, H, n, d, code, dev, probe, part="scratch") if separate_scratch else None
     O = torch.empty_like(Q)

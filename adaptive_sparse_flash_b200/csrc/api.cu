@@ -119,8 +119,9 @@ entmax_status check_dims(int B, int H, int n, int d, entmax_dtype dt, const entm
 }
 
 // Workspace, in two parts.
-//   saved   - what the backward needs from the forward: U V (fp32 [BH][n][d]), sum u ([BH][n]) and the
-//             transposed mask;
+//   saved   - what the backward needs from the forward: sum u ([BH][n]), the transposed mask and, for the
+//             bf16 and fp32 kernels (not the fp16 family, whose dQ kernel forms delta itself), U V (fp32
+//             [BH][n][d]);
 //   scratch - per call: delta and the row statistic padded to whole 64-row blocks ([BH][ceil(n/64)*64]) for
 //             the backward, the range words, and the fp16 operand copies of Q, K, V, dO (f16.cu).
 // With one buffer (opts->scratch NULL) the scratch part follows the saved part, and a backward reuses the
@@ -141,14 +142,17 @@ struct Workspace {
     bool separate;      // scratch in its own buffer
 };
 
-Workspace layout(const Dims& D, void* base, void* scratch) {
+Workspace layout(const Dims& D, void* base, void* scratch, bool with_obar) {
     const size_t rows = (size_t)D.B * D.H * D.n;
     const size_t rows_pad = (size_t)D.B * D.H * (size_t)((D.n + 63) / 64) * 64;
     Workspace w;
     char* p = static_cast<char*>(base);
     size_t off = 0;
-    w.obar = reinterpret_cast<float*>(p + off);
-    off = align256(off + rows * D.d * sizeof(float));
+    w.obar = nullptr;
+    if (with_obar) {
+        w.obar = reinterpret_cast<float*>(p + off);
+        off = align256(off + rows * D.d * sizeof(float));
+    }
     w.sum_u = reinterpret_cast<float*>(p + off);
     off = align256(off + rows * sizeof(float));
     w.maskT = reinterpret_cast<uint32_t*>(p + off);
@@ -172,11 +176,11 @@ Workspace layout(const Dims& D, void* base, void* scratch) {
     return w;
 }
 
-entmax_status check_workspace(const Dims& D, const entmax_opts* o, Workspace* w) {
+entmax_status check_workspace(const Dims& D, const entmax_opts* o, Workspace* w, bool with_obar) {
     if (!o || !o->workspace) return ENTMAX_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(o->workspace) & 255u) != 0) return ENTMAX_ERR_ALIGN;
     if (o->scratch && (reinterpret_cast<uintptr_t>(o->scratch) & 255u) != 0) return ENTMAX_ERR_ALIGN;
-    *w = layout(D, o->workspace, o->scratch);
+    *w = layout(D, o->workspace, o->scratch, with_obar);
     if (o->scratch) {
         if (o->workspace_bytes < w->saved_bytes || o->scratch_bytes < w->scratch_bytes) return ENTMAX_ERR_WORKSPACE;
     } else if (o->workspace_bytes < w->saved_bytes + w->scratch_bytes) {
@@ -186,6 +190,14 @@ entmax_status check_workspace(const Dims& D, const entmax_opts* o, Workspace* w)
 }
 
 inline entmax_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ENTMAX_OK : ENTMAX_ERR_CUDA; }
+
+bool use_f16_path(int d, float alpha, int nw, int bins);
+
+// U V is part of the saved workspace unless the fp16 family serves the call (bf16, d = 64, alpha <= 2).
+// alpha <= 1 (unknown, for sizing) keeps it.
+inline bool needs_obar(const Dims& D, float alpha, entmax_dtype dt) {
+    return !(dt == ENTMAX_BF16 && alpha > 1.0f && use_f16_path(D.d, alpha, D.nw, D.bins));
+}
 
 int num_sms() {
     static int cache[64] = {0};
@@ -203,7 +215,7 @@ int num_sms() {
 // its shared memory (which grows with the number of mask words per row and with the histogram size) fits;
 // the backward follows the forward's choice (it reads the forward's fp16 copies).
 constexpr size_t kMaxDynSmem = 232448;
-inline bool use_f16_path(int d, float alpha, int nw, int bins) {
+bool use_f16_path(int d, float alpha, int nw, int bins) {
     return d == 64 && alpha <= 2.0f && fwd_h_smem_bytes(nw, bins) <= kMaxDynSmem;
 }
 
@@ -234,20 +246,20 @@ EATTN_API const char* entmax_status_str(entmax_status s) {
 EATTN_API size_t entmax_attn_workspace_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts) {
     Dims D;
     if (check_dims(B, H, n, d, dt, opts, &D) != ENTMAX_OK) return 0;
-    const Workspace w = layout(D, nullptr, nullptr);
+    const Workspace w = layout(D, nullptr, nullptr, needs_obar(D, opts ? opts->alpha : 0.0f, dt));
     return w.saved_bytes + w.scratch_bytes;
 }
 
 EATTN_API size_t entmax_attn_saved_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts) {
     Dims D;
     if (check_dims(B, H, n, d, dt, opts, &D) != ENTMAX_OK) return 0;
-    return layout(D, nullptr, nullptr).saved_bytes;
+    return layout(D, nullptr, nullptr, needs_obar(D, opts ? opts->alpha : 0.0f, dt)).saved_bytes;
 }
 
 EATTN_API size_t entmax_attn_scratch_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts) {
     Dims D;
     if (check_dims(B, H, n, d, dt, opts, &D) != ENTMAX_OK) return 0;
-    return layout(D, nullptr, nullptr).scratch_bytes;
+    return layout(D, nullptr, nullptr, false).scratch_bytes;
 }
 
 EATTN_API entmax_status entmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* tau,
@@ -260,7 +272,7 @@ EATTN_API entmax_status entmax_attn_fwd(const void* Q, const void* K, const void
     if (st != ENTMAX_OK) return st;
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return ENTMAX_ERR_ALIGN;
     Workspace ws;
-    if ((st = check_workspace(D, opts, &ws)) != ENTMAX_OK) return st;
+    if ((st = check_workspace(D, opts, &ws, needs_obar(D, alpha, dt))) != ENTMAX_OK) return st;
     int* status = status_ptr();
     if (!status) return ENTMAX_ERR_CUDA;
 
@@ -342,7 +354,7 @@ entmax_status bwd_common(const void* Q, const void* K, const void* V, const void
         !aligned16(dK) || !aligned16(dV))
         return ENTMAX_ERR_ALIGN;
     Workspace ws;
-    if ((st = check_workspace(D, opts, &ws)) != ENTMAX_OK) return st;
+    if ((st = check_workspace(D, opts, &ws, !softmax && needs_obar(D, alpha, dt))) != ENTMAX_OK) return st;
     int* status = status_ptr();
     if (!status) return ENTMAX_ERR_CUDA;
     const float scale = opts->scale != 0.0f ? opts->scale : 1.0f / sqrtf((float)d);
@@ -439,7 +451,7 @@ EATTN_API entmax_status softmax_attn_fwd(const void* Q, const void* K, const voi
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     TrailScope trail(opts, s);
     Workspace ws;
-    if (d == 64 && opts && opts->workspace && check_workspace(D, opts, &ws) == ENTMAX_OK) {
+    if (d == 64 && opts && opts->workspace && check_workspace(D, opts, &ws, false) == ENTMAX_OK) {
         // fp16 path: copies of Q, K, V in the workspace
         F16Job job;
         memset(&job, 0, sizeof(job));

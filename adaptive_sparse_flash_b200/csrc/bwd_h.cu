@@ -508,16 +508,31 @@ constexpr uint32_t qOffO = kTile;
 constexpr uint32_t qOffSt = 2 * kTile;
 constexpr uint32_t qOffBar = qOffSt + NST * kStageQ;
 
-template <int KIND>
+// Three forms, one launch each in entmax mode, of which the range word of K (dq_one_term) lets exactly the
+// needed ones work and the others return at once (uniform over the CTA, before any barrier or TMEM use):
+//   MODE kDqAB    - keys of unit scale: dQ = scale (A - delta B) with A = (u g) K and B = u K in two
+//                   accumulators, delta from this kernel's own row sums (one fp16 term each);
+//   MODE kDqDelta - larger keys, first: the delta pass (row sums only, no dQ product);
+//   MODE kDqPlain - larger keys, second, and the softmax baseline: dS = u (g - delta) with delta from the
+//                   delta pass (entmax) or from bwd_pre (softmax), one or two fp16 terms.
+enum DqMode : int { kDqPlain = 0, kDqAB = 1, kDqDelta = 2 };
+
+template <int KIND, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_h_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const BwdArgs a, float* __restrict__ delta_pad, const float* __restrict__ stat_pad) {
+    constexpr bool ENT = KIND != kSoftmaxH;
+    constexpr bool delta_only = MODE == kDqDelta;
+    constexpr bool ab = MODE == kDqAB;
+    static_assert(ENT || MODE == kDqPlain, "the softmax baseline takes its delta from bwd_pre");
+    const bool one = dq_one_term(a);
+    if (ENT && (ab != one)) return;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* smem = align_smem_1024(smem_raw);
     Bars& bb = *reinterpret_cast<Bars*>(smem + qOffBar);
-    float* xsum = reinterpret_cast<float*>(&bb + 1);          // [TM]: warpgroup 1's row sums of dS~
-    uint32_t* vis = reinterpret_cast<uint32_t*>(xsum + TM);     // [nw] key blocks to visit
+    float* xsum = reinterpret_cast<float*>(&bb + 1);             // [2][TM]: each warpgroup's row sums of u g
+    uint32_t* vis = reinterpret_cast<uint32_t*>(xsum + 2 * TM);  // [nw] key blocks to visit
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qt = (int)gridDim.x - 1 - (int)blockIdx.x;
@@ -608,6 +623,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_ss(tmem + 128u * g + 64, sdesc_at(kDescK, sO + kk * 32), sdesc_at(kDescK, vb + kk * 32), idS,
                            kk > 0);
                 mma_commit(&bb.d_full[g]);
+                if constexpr (delta_only) mma_commit(&bb.q_empty[st]);  // no dQ product reads this K block
             }
             mma_commit(&bb.drain[0]);
             wait_drain(&bb.drain[0], 0, 200000000ull);
@@ -615,25 +631,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 10) {
         if (lane == 0) {
             constexpr uint32_t idG = idesc_f16_f32(TM, D, false, true);  // dS K (MN-major B)
-            const bool one = dq_one_term(a);
             bool ok = true;
-            for (int t = 0; t < T && ok; ++t) {
+            for (int t = 0; t < T && ok && !delta_only; ++t) {
                 const int g = t & 1;
                 const uint32_t j = (uint32_t)(t >> 1), st = (uint32_t)t % NST;
                 if (!(ok = wait_bounded(&bb.a_full[g], j & 1, abort_flag, a.status, true))) break;
                 tc_fence_after();
                 const uint32_t kb = sSt + st * kStageQ;
-                const uint32_t ta = tmem + 256u + 64u * g;  // dS hi, lo
+                const uint32_t ta = tmem + 256u + 64u * g;  // [dS hi | dS lo], or [u g | u] (ab)
 #pragma unroll
                 for (int kk = 0; kk < TB / 16; ++kk) {
                     const uint64_t dk = sdesc_at(kDescMN, kb + kk * 2048);
-                    mma_ts(tmem + 384, ta + 8 * kk, dk, idG, (t == 0 && kk == 0) ? 0u : 1u);
-                    if (!one) mma_ts(tmem + 384, ta + 32 + 8 * kk, dk, idG, 1u);
+                    const uint32_t acc = (t == 0 && kk == 0) ? 0u : 1u;
+                    mma_ts(tmem + 384, ta + 8 * kk, dk, idG, acc);
+                    if (ab) mma_ts(tmem + 448, ta + 32 + 8 * kk, dk, idG, acc);
+                    else if (!one) mma_ts(tmem + 384, ta + 32 + 8 * kk, dk, idG, 1u);
                 }
                 mma_commit(&bb.a_empty[g]);
                 mma_commit(&bb.q_empty[st]);
             }
-            if (ok && T > 0) mma_commit(&bb.acc_full);
+            if (ok && T > 0 && !delta_only) mma_commit(&bb.acc_full);
             mma_commit(&bb.drain[1]);
             wait_drain(&bb.drain[1], 0, 200000000ull);
         }
@@ -644,10 +661,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool qvalid = row < a.n;
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const Scales sc = make_scales(a);
-        const bool one = dq_one_term(a);
         const float tau = stat_pad[(size_t)bh * npad + min(row, npad - 1)];
-        const float dl = delta_pad[(size_t)bh * npad + min(row, npad - 1)] * sc.dl;
-        float rs = 0.f;  // this warpgroup's share of the row sum of u (g - d~), in dP units
+        // delta in dP units: from bwd_pre (softmax) or the delta pass (entmax, larger keys); unused otherwise
+        const float dl = (ENT && (ab || delta_only)) ? 0.f : delta_pad[(size_t)bh * npad + min(row, npad - 1)] * sc.dl;
+        float rs = 0.f;  // this warpgroup's share of the row sum of u g, in dP units (entmax, ab / delta pass)
         bool ok = true;
         int t = 0;
         uint32_t j = 0;
@@ -696,16 +713,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bb.d_empty[g]);
+                if constexpr (delta_only) {
+#pragma unroll
+                    for (int c = 0; c < TB; ++c) rs = fmaf(sv[c], dp[c], rs);
+                    ++j;
+                    continue;
+                }
 #pragma unroll
                 for (int c = 0; c < TB; ++c) {
                     const float e = sv[c] * (dp[c] - dl);
-                    if constexpr (KIND != kSoftmaxH) rs += e;
+                    if (ab) rs += e;
                     dp[c] = e * sc.ds;
                 }
                 ok = __all_sync(0xffffffffu, wait_bounded(&bb.a_empty[g], (j & 1) ^ 1, abort_flag, a.status));
                 if (!ok) break;
                 const uint32_t ta = lane_base + 256u + 64u * g;
-                if (one) {
+                if (ab) {
+                    // [u g | u], one fp16 term each (keys of unit scale), 32 keys at a time
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        uint32_t wa[16], wu[16];
+#pragma unroll
+                        for (int c = 0; c < 32; c += 2) {
+                            wa[c / 2] = pack_half2(dp[32 * h + c], dp[32 * h + c + 1]);
+                            wu[c / 2] = pack_half2(sv[32 * h + c], sv[32 * h + c + 1]);
+                        }
+                        tmem_st16(ta + 16 * h, wa);
+                        tmem_st16(ta + 32 + 16 * h, wu);
+                    }
+                } else if (one) {
                     uint32_t w32[32];
 #pragma unroll
                     for (int c = 0; c < TB; c += 2) w32[c / 2] = pack_half2(dp[c], dp[c + 1]);
@@ -728,36 +764,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++j;
             }
         }
-        if (g == 1) xsum[r] = rs;
+        xsum[g * TM + r] = rs;
         ok = !bar_or256(!ok || *abort_flag != 0);
-        if constexpr (KIND != kSoftmaxH) {
-            // the exact delta of this row, for the dK / dV kernel that runs next
-            if (ok && g == 0 && qvalid) {
-                const float s_u = a.sum_u[(size_t)bh * a.n + row];
-                const float corr = s_u > 0.f ? (rs + xsum[r]) / s_u : 0.f;
-                delta_pad[(size_t)bh * npad + row] = (dl + corr) / sc.dl;
-            }
+        // entmax: delta = sum u g / sum u of this row (sum u from the forward, over the same u: both passes
+        // form x = fma(s, cz, -tau) from the same score tile), in dP units; written back for the dK / dV kernel
+        float dlx = 0.f;
+        if (ENT && (ab || delta_only)) {
+            const float s_u = qvalid ? a.sum_u[(size_t)bh * a.n + row] : 0.f;
+            dlx = s_u > 0.f ? (xsum[r] + xsum[TM + r]) / s_u : 0.f;
+            if (ok && g == 0 && qvalid) delta_pad[(size_t)bh * npad + row] = dlx / sc.dl;
         }
-        if (T > 0 && ok) ok = __all_sync(0xffffffffu, wait_bounded(&bb.acc_full, 0, abort_flag, a.status));
-        ok = !bar_or256(!ok || *abort_flag != 0);
-        // warpgroup g writes columns 32 g .. 32 g + 31 of dQ
-        float* dQ = static_cast<float*>(a.dQ) + ((size_t)bh * a.n + row) * D + 32 * g;
-        if (ok && T > 0) {
-            tc_fence_after();
-            __syncwarp();
-            uint32_t qq[32];
-            tmem_ld32(lane_base + 384u + 32u * g, qq);
-            tmem_ld_wait();
-            if (qvalid) {
+        if constexpr (!delta_only) {
+            if (T > 0 && ok) ok = __all_sync(0xffffffffu, wait_bounded(&bb.acc_full, 0, abort_flag, a.status));
+            ok = !bar_or256(!ok || *abort_flag != 0);
+            // warpgroup g writes columns 32 g .. 32 g + 31 of dQ; ab: dQ = scale (A - delta B)
+            float* dQ = static_cast<float*>(a.dQ) + ((size_t)bh * a.n + row) * D + 32 * g;
+            if (ok && T > 0) {
+                tc_fence_after();
+                __syncwarp();
+                uint32_t qq[32];
+                tmem_ld32(lane_base + 384u + 32u * g, qq);
+                tmem_ld_wait();
+                if (ab) {
+                    uint32_t qb[32];
+                    tmem_ld32(lane_base + 448u + 32u * g, qb);
+                    tmem_ld_wait();
+                    const float db = dlx * sc.ds;
 #pragma unroll
-                for (int q = 0; q < 32; q += 4)
-                    *reinterpret_cast<float4*>(dQ + q) =
-                        make_float4(sc.dq * __uint_as_float(qq[q]), sc.dq * __uint_as_float(qq[q + 1]),
-                                    sc.dq * __uint_as_float(qq[q + 2]), sc.dq * __uint_as_float(qq[q + 3]));
+                    for (int q = 0; q < 32; ++q)
+                        qq[q] = __float_as_uint(fmaf(-db, __uint_as_float(qb[q]), __uint_as_float(qq[q])));
+                }
+                if (qvalid) {
+#pragma unroll
+                    for (int q = 0; q < 32; q += 4)
+                        *reinterpret_cast<float4*>(dQ + q) =
+                            make_float4(sc.dq * __uint_as_float(qq[q]), sc.dq * __uint_as_float(qq[q + 1]),
+                                        sc.dq * __uint_as_float(qq[q + 2]), sc.dq * __uint_as_float(qq[q + 3]));
+                }
+                tc_fence_before();
+            } else if (ok && qvalid) {
+                for (int c = 0; c < 32; c += 4) *reinterpret_cast<float4*>(dQ + c) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            tc_fence_before();
-        } else if (ok && qvalid) {
-            for (int c = 0; c < 32; c += 4) *reinterpret_cast<float4*>(dQ + c) = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     }
     tc_fence_before();
@@ -782,16 +829,28 @@ cudaError_t launch_h_t(const BwdArgs& a, float* delta_pad, float* stat_pad, cuda
     if ((e = make_tmap_f16(&tk64, a.Kh, BH, a.n, D, TB)) != cudaSuccess) return e;
     if ((e = make_tmap_f16(&tv64, a.Vh, BH, a.n, D, TB)) != cudaSuccess) return e;
     const int ntiles = (a.n + TM - 1) / TM;
-    // dQ first: it writes the exact delta of every row (entmax), which the dK / dV kernel then reads
+    // dQ first: it writes the exact delta of every row (entmax), which the dK / dV kernel then reads. In entmax
+    // mode a delta pass of the same kernel runs before it; it does work only for keys of more than unit scale.
     {
-        const size_t bytes = 1024 + qOffBar + sizeof(Bars) + TM * sizeof(float) + (size_t)a.nw * 4;
+        const size_t bytes = 1024 + qOffBar + sizeof(Bars) + 2 * TM * sizeof(float) + (size_t)a.nw * 4;
         if (bytes > 232448) return cudaErrorInvalidConfiguration;
-        auto kern = bwd_h_dq_kernel<KIND>;
-        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
-            return e;
-        launch_mark(stream);
-        kern<<<dim3(ntiles, BH), kThreads, bytes, stream>>>(tq128, tk64, tv64, tdo128, a, delta_pad, stat_pad);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        using Kern = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, BwdArgs, float*, const float*);
+        Kern kerns[3];
+        int nk = 0;
+        if (KIND != kSoftmaxH) {
+            kerns[nk++] = bwd_h_dq_kernel<KIND, (KIND != kSoftmaxH ? kDqAB : kDqPlain)>;
+            kerns[nk++] = bwd_h_dq_kernel<KIND, (KIND != kSoftmaxH ? kDqDelta : kDqPlain)>;
+        }
+        kerns[nk++] = bwd_h_dq_kernel<KIND, kDqPlain>;
+        for (int i = 0; i < nk; ++i) {
+            if ((e = cudaFuncSetAttribute(kerns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) !=
+                cudaSuccess)
+                return e;
+            launch_mark(stream);
+            kerns[i]<<<dim3(ntiles, BH), kThreads, bytes, stream>>>(tq128, tk64, tv64, tdo128, a, delta_pad,
+                                                                     stat_pad);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
     }
     {
         const size_t bytes = 1024 + kvOffBar + sizeof(Bars) + (size_t)a.nwq * 4;

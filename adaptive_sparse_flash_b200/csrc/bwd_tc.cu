@@ -9,7 +9,8 @@
 // and "Bit-Packed Block Mask"; the largest gain is in the backward, section 4 "Ergebnisse").
 //
 // Kernels (all 192 threads: warps 0-3 compute, warp 4 MMA issue, warp 5 TMA issue):
-//   bwd_pre    delta per query row, and padded copies of the row statistics for bulk copies;
+//   bwd_pre    delta per query row (from U V; 0 when the caller passes no U V, as the fp16 backward does,
+//              whose dQ kernel forms delta itself), and padded copies of the row statistics for bulk copies;
 //   bwd_dkdv   one CTA per 128-key tile: walks the tile's query blocks (transposed mask), recomputes
 //              S^T = K Q^T and dP^T = V dO^T into TMEM, forms P^T and dS^T (thread = key row) in
 //              shared memory, accumulates dV += P^T dO and dK += dS^T Q in TMEM;
@@ -119,7 +120,8 @@ __global__ void bwd_pre_kernel(const BwdArgs a, float* __restrict__ delta_pad, f
         if (a.softmax) {
             const __nv_bfloat16* O = static_cast<const __nv_bfloat16*>(a.O) + base;
             for (int c = lane; c < D; c += 32) acc = fmaf(__bfloat162float(dO[c]), __bfloat162float(O[c]), acc);
-        } else {
+        } else if (a.obar) {
+            // the bf16 family's delta from U V; the fp16 backward forms delta in its dQ kernel (obar NULL)
             const float* Ob = a.obar + base;
             for (int c = lane; c < D; c += 32) acc = fmaf(__bfloat162float(dO[c]), Ob[c], acc);
         }

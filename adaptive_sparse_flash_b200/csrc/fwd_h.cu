@@ -6,22 +6,21 @@
 //                   and reads TMEM lane r; the two warpgroups take alternate key blocks of every sweep;
 //   warp 8          S issue (one thread): S = Q K^T from shared memory into three TMEM buffers per
 //                   warpgroup;
-//   warp 10         P V issue (one thread): O += P V and Obar += U V with P and U stored by the compute
-//                   warps into the TMEM columns of the S tile they came from. Two issuing threads keep the
-//                   tensor pipe fed: each waits only on its own barriers, in block order;
+//   warp 10         P V issue (one thread): O += P V with P stored by the compute warps into the TMEM
+//                   columns of the S tile it came from. Two issuing threads keep the tensor pipe fed: each
+//                   waits only on its own barriers, in block order;
 //   warp 9          TMA issue (one thread): Q once, K blocks of 64 keys and, in P V sweeps, V blocks.
 //
-// P and U lie in [0, 1] for alpha <= 2 and each enters its product as one fp16 term (11 significant bits;
-// bf16 would need a two-term split). U V only gives the backward a first estimate of
-// delta = dO . (U V) / sum u for its dQ kernel, which then accumulates the exact delta from fp32 u and g
-// (bwd_h.cu); so one term is enough here. P and U of a 64-key block fit the 64 columns of its S tile. A
-// new S tile goes into a buffer only after the P V products that read its previous P and U have
-// completed (a commit barrier per buffer), and the MMA thread waits for all P V products at the end of a
-// P V sweep: MMAs into different accumulators are not ordered by issue alone.
+// P lies in [0, 1] for alpha <= 2 and enters P V as one fp16 term (11 significant bits; bf16 would need a
+// two-term split). The backward needs no product of u with V from the forward: its dQ kernel forms
+// delta = sum u g / sum u itself (bwd_h.cu), so this kernel writes only O, tau, sum u and the mask. P of a
+// 64-key block fits the first 32 columns of its S tile. A new S tile goes into a buffer only after the P V
+// products that read its previous P have completed (a commit barrier per buffer), and the MMA thread waits
+// for all P V products at the end of a P V sweep: MMAs into different accumulators are not ordered by issue
+// alone.
 //
-// TMEM columns (512): S buffer b (of three) of warpgroup g at 64 (3 g + b), holding P (first 32 columns)
-// and U (next 32; K step kk of 16 keys is columns 8 kk .. 8 kk + 7 of each) in P V sweeps; O at 384, U V at
-// 448.
+// TMEM columns (512): S buffer b (of three) of warpgroup g at 64 (3 g + b), holding P in its first 32
+// columns (K step kk of 16 keys is columns 8 kk .. 8 kk + 7) in P V sweeps; O at 384.
 //
 // Sweeps follow the plan protocol of the bf16 forward (fwd_tc.cu): before each sweep the compute warps
 // publish its kind and its set of key blocks, which the issuing warps follow.
@@ -32,7 +31,7 @@
 //             bins those rows' entries into their histograms with the window fixed by the final max;
 //   refine  - candidate blocks: solver sums at the current tau (partial sums of the two warpgroups are
 //             combined by warpgroup 0, which owns the solver state of each row);
-//   P V     - candidate blocks: p and u to TMEM for the P V and U V MMAs, exact block mask, sum check.
+//   P V     - candidate blocks: p to TMEM for the P V MMAs, exact block mask, sum check.
 // (AdaSplash-2, gist.science (de), section 2: histogram initialisation, hybrid solver, bit-packed block
 // mask, only nonzero blocks processed.)
 #include <cuda.h>
@@ -89,7 +88,6 @@ struct HCfg {
 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 384;
-constexpr uint32_t kColOb = 448;
 
 // exchange rows of Small::xf
 enum : int {
@@ -107,8 +105,8 @@ struct Small {
     uint64_t k_full[NKS_MAX], k_empty[NKS_MAX];
     uint64_t v_full[NVS], v_empty[NVS];
     uint64_t s_full[2][NSB], s_empty[2][NSB];  // [warpgroup][buffer]
-    uint64_t pv_free[2][NSB];                  // P V products that read a buffer's P and U have completed
-    uint64_t pu_full[2][NSB];                  // a buffer's P and U are stored (one barrier per buffer, so
+    uint64_t pv_free[2][NSB];                  // P V products that read a buffer's P have completed
+    uint64_t pu_full[2][NSB];                  // a buffer's P is stored (one barrier per buffer, so
                                            // that no barrier runs two phases ahead of its waiter)
     uint64_t o_full;
     uint64_t ctrl;
@@ -336,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!(ok = wait_bounded(&sm.ctrl, sw & 1, abort_flag, a.status, true))) break;
                 const int kind = sm.plan_kind[sw & 1];
                 if (after_pv) {
-                    // every P V of the last P V sweep complete before a buffer holding P / U is overwritten
+                    // every P V of the last P V sweep complete before a buffer holding P is overwritten
                     if (!(ok = wait_bounded(&sm.o_full, (npv - 1) & 1, abort_flag, a.status, true))) break;
                     after_pv = false;
                 }
@@ -406,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t b = sn % NSB;
                     const uint32_t bi = NSB * g + b;
                     const uint32_t vs = vc % NVS;
-                    // k P V products on a buffer so far: its P / U store number k + 1 completes phase k
+                    // k P V products on a buffer so far: its P store number k + 1 completes phase k
                     if (!(ok = wait_bounded(&sm.pu_full[g][b], ((ppar >> bi) & 1u) ^ 1u, abort_flag, a.status, true))) break;
                     if (!(ok = wait_bounded(&sm.v_full[vs], (vc / NVS) & 1, abort_flag, a.status, true))) break;
                     tc_fence_after();
@@ -417,7 +415,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint64_t dv = sdesc_at(kDescMN, vbase + kk * 2048);
                         const uint32_t acc = (tp == 0 && kk == 0) ? 0u : 1u;
                         mma_ts(tmem + kColO, tpu + 8 * kk, dv, idPV, acc);
-                        mma_ts(tmem + kColOb, tpu + 32 + 8 * kk, dv, idPV, acc);
                     }
                     mma_commit(&sm.pv_free[g][b]);
                     mma_commit(&sm.v_empty[vs]);
@@ -735,7 +732,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ++refine;
         };
 
-        // ---- P V sweep: p, u to TMEM for the P V / U V MMAs, exact mask, sum check ----
+        // ---- P V sweep: p to TMEM for the P V MMAs, exact mask, sum check ----
         float Su = 0.f;
         auto pv_sweep = [&]() -> bool {
             if (g == 0) {
@@ -760,51 +757,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float amax = group_max();
                     const bool keep = sp.cz * amax > lo0;
                     const bool nz = fmaf(amax, sp.cz, -t) > 0.f;
-                    // one branch-free pass over the block, 32 keys at a time: p and u of each key, packed as
-                    // fp16 pairs into the columns of the S tile just read (this warpgroup's own buffer), P in
-                    // the first 32 columns and U in the next 32. The solver sums ride along in warps that hold
-                    // a row whose tau still needs the check.
+                    // one branch-free pass over the block, 32 keys at a time: p of each key, packed as fp16
+                    // pairs into the first 32 columns of the S tile just read (this warpgroup's own buffer).
+                    // The solver sums (and u) ride along in warps that hold a row whose tau still needs the
+                    // check.
                     const uint32_t tp = lane_base + colS;
                     auto pu_pass = [&](auto with_sums) {
                         constexpr bool SUMS = decltype(with_sums)::value;
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
-                            uint32_t wp[16], wu[16];
+                            uint32_t wp[16];
 #pragma unroll
                             for (int c = 0; c < 32; c += 2) {
-                                float p2[2], u2[2];
+                                float p2[2];
 #pragma unroll
                                 for (int h2 = 0; h2 < 2; ++h2) {
                                     const float x = fmaf(vbuf[32 * h + c + h2], sp.cz, -t);
-                                    float pp, uu;
+                                    float pp;
                                     if constexpr (KIND == kAlpha15) {
-                                        uu = fmaxf(x, 0.f);
+                                        const float uu = fmaxf(x, 0.f);
                                         pp = uu * uu;
-                                        if constexpr (SUMS) F2 += x > 0.f ? 1.f : 0.f;
+                                        if constexpr (SUMS) {
+                                            F2 += x > 0.f ? 1.f : 0.f;
+                                            Sq += uu;
+                                        }
                                     } else if constexpr (KIND == kAlpha2) {
                                         pp = fmaxf(x, 0.f);
-                                        uu = x > 0.f ? 1.f : 0.f;
+                                        if constexpr (SUMS) Sq += x > 0.f ? 1.f : 0.f;
                                     } else {
                                         const bool pos = x > 0.f;
                                         const float xs = pos ? x : 1.f;
                                         const float u1 = exp2f((sp.k - 1.f) * __log2f(xs));
-                                        uu = pos ? u1 : 0.f;
+                                        const float uu = pos ? u1 : 0.f;
                                         pp = uu * xs;
-                                        if constexpr (SUMS) F2 += pos ? __fdividef(u1, xs) : 0.f;
+                                        if constexpr (SUMS) {
+                                            F2 += pos ? __fdividef(u1, xs) : 0.f;
+                                            Sq += uu;
+                                        }
                                     }
                                     if constexpr (SUMS) {
                                         Sp += pp;
-                                        Sq += uu;
                                         Sn += x > 0.f ? 1u : 0u;
                                     }
                                     p2[h2] = pp;
-                                    u2[h2] = uu;
                                 }
                                 wp[c / 2] = pack_half2(p2[0], p2[1]);
-                                wu[c / 2] = pack_half2(u2[0], u2[1]);
                             }
                             tmem_st16(tp + 16 * h, wp);
-                            tmem_st16(tp + 32 + 16 * h, wu);
                         }
                     };
                     if (need_sums) pu_pass(std::true_type{});
@@ -861,35 +860,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             while (ok && refine < kMaxSweeps && bar_or256(g == 0 && !s.done)) refine_sweep();
         }
 
-        // ---- wait for the last P V MMAs, then write O (warpgroup 0), U V (warpgroup 1), tau, sum u ----
+        // ---- wait for the last P V MMAs, then write O (warpgroup g: columns 32 g .. 32 g + 31), tau, sum u ----
         if (ok) ok = __all_sync(0xffffffffu, wait_bounded(&sm.o_full, (pv - 1) & 1, abort_flag, a.status));
         ok = !bar_or256(!ok || *abort_flag != 0);
         if (ok) {
             tc_fence_after();
             __syncwarp();
-            uint32_t o[64];
-            const uint32_t col = g == 0 ? kColO : kColOb;
-            tmem_ld32(lane_base + col, o);
-            tmem_ld32(lane_base + col + 32, o + 32);
+            uint32_t o[32];
+            tmem_ld32(lane_base + kColO + 32u * g, o);
             tmem_ld_wait();
             if (valid) {
-                if (g == 0) {
-                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + (head + row) * D);
+                uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + (head + row) * D + 32 * g);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float* f = reinterpret_cast<const float*>(o + 8 * i);
-                        dst[i] = make_uint4(pack_bf16x2(f[0] * vscale, f[1] * vscale),
-                                            pack_bf16x2(f[2] * vscale, f[3] * vscale),
-                                            pack_bf16x2(f[4] * vscale, f[5] * vscale),
-                                            pack_bf16x2(f[6] * vscale, f[7] * vscale));
-                    }
-                } else {
-                    float4* dob = reinterpret_cast<float4*>(a.obar + (head + row) * D);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float* f = reinterpret_cast<const float*>(o + 4 * i);
-                        dob[i] = make_float4(f[0] * vscale, f[1] * vscale, f[2] * vscale, f[3] * vscale);
-                    }
+                for (int i = 0; i < 4; ++i) {
+                    const float* f = reinterpret_cast<const float*>(o + 8 * i);
+                    dst[i] = make_uint4(pack_bf16x2(f[0] * vscale, f[1] * vscale),
+                                        pack_bf16x2(f[2] * vscale, f[3] * vscale),
+                                        pack_bf16x2(f[4] * vscale, f[5] * vscale),
+                                        pack_bf16x2(f[6] * vscale, f[7] * vscale));
                 }
             }
             tc_fence_before();

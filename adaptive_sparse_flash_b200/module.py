@@ -24,9 +24,9 @@ class EntmaxAttnFunction(torch.autograd.Function):
     """O = alpha-entmax(scale Q K^T) V for bf16 [B, H, n, d] tensors on a CUDA device (d in {64, 128}).
 
     Besides q, k, v and O, the forward keeps tau, the block mask and the saved part of the library's
-    workspace (U V in fp32, sum u, the transposed mask) for the backward; the fp16 operand copies live in a
-    per-call scratch buffer, so they are not activation memory. Gradients come back in the inputs' dtype
-    (the library computes them in fp32).
+    workspace for the backward: sum u and the transposed mask (plus U V in fp32 where the bf16 kernels serve
+    the call, d = 128 or alpha > 2); the fp16 operand copies live in a per-call scratch buffer, so they are
+    not activation memory. Gradients come back in the inputs' dtype (the library computes them in fp32).
     """
 
     @staticmethod

@@ -35,9 +35,12 @@ METRIC = "α-entmax attn fwd+bwd effective TFLOP/s at n=16k vs sparsity; % bf16 
 # kernels of one call on the fp16 operand path (d = 64, alpha <= 2), in launch order (include/entmax_attn.h,
 # "Per-kernel timing"); the L2 flush between steps is a torch fill and is not counted
 FWD_KERNELS = ("to_f16_pass1", "to_f16_pass2", "fwd_h_kernel", "mask_transpose_kernel")
-BWD_KERNELS = ("to_f16_pass1", "to_f16_pass2", "bwd_pre_kernel", "bwd_h_dq_kernel", "bwd_h_dkdv_kernel")
+# the backward's dQ kernel has three launches, of which K's range lets one route work: for unit-scale keys (the
+# bench) the first; for larger keys the delta pass and the plain pass. The others return at once.
+BWD_KERNELS = ("to_f16_pass1", "to_f16_pass2", "bwd_pre_kernel", "bwd_h_dq_kernel", "bwd_h_dq_delta_pass",
+               "bwd_h_dq_plain_pass", "bwd_h_dkdv_kernel")
 SM_FWD_KERNELS = ("to_f16_pass1", "to_f16_pass2", "softmax_fwd_h_kernel")
-SM_BWD_KERNELS = BWD_KERNELS
+SM_BWD_KERNELS = ("to_f16_pass1", "to_f16_pass2", "bwd_pre_kernel", "bwd_h_dq_kernel", "bwd_h_dkdv_kernel")
 LAUNCHES_PER_STEP = len(FWD_KERNELS) + len(BWD_KERNELS)
 WORKLOAD = (f"alpha-entmax attention fwd+bwd, B={B} H={H} n={N} d={D} bf16 causal alpha={ALPHA}, "
             f"keys clustered on {CENTRES} centres (noise 0.3), queries {BETA_Q:g} x centre + noise")
@@ -87,7 +90,7 @@ def kernel_flops(n, d, heads, nnz_blocks):
 
     Entmax: the forward owns the dense Q K^T pass and the nonzero-block P V product; of the five backward
     products per nonzero block, the dK / dV kernel owns S, dP, dV and dK, the dQ kernel owns dQ (its
-    recomputed S and dP are not counted). Dense softmax baseline: two products over every causal entry in
+    recomputed S and dP, and its split of dQ into (u g) K and u K, are not counted). Dense softmax baseline: two products over every causal entry in
     the forward (S, P V), four in the dK / dV kernel and one in the dQ kernel."""
     qk = 2.0 * d * n * (n + 1) / 2 * heads
     blk = 2.0 * d * BLOCK * BLOCK * nnz_blocks

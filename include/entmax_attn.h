@@ -88,11 +88,15 @@ typedef struct {
     void* scratch;          /* optional per-call scratch (>= entmax_attn_scratch_size() bytes, 256-aligned);
                                NULL: the scratch lies inside the workspace (see "Workspace" below)    */
     size_t scratch_bytes;
+    float alpha;            /* sizing only: the alpha the workspace will serve (0: any; see below)    */
 } entmax_opts;
 
 /* Workspace. The library's device scratch has two parts:
- *   saved   - written by the forward and read by its backward: U V (fp32 [B,H,n,d]), sum u (fp32 [B,H,n])
- *             and the transposed block mask; entmax_attn_saved_size() bytes;
+ *   saved   - written by the forward and read by its backward: sum u (fp32 [B,H,n]), the transposed block
+ *             mask and, unless the fp16 kernels serve the call (bf16, d = 64, alpha <= 2), U V (fp32
+ *             [B,H,n,d]); entmax_attn_saved_size() bytes. The size functions leave U V out only when
+ *             opts->alpha names an alpha in (1, 2] (with d = 64, bf16); a workspace sized without U V
+ *             makes calls with another alpha return ENTMAX_ERR_WORKSPACE;
  *   scratch - used within one call: the fp16 operand copies of Q, K, V, dO, the padded per-row delta and
  *             row statistic, range words; entmax_attn_scratch_size() bytes.
  * With opts->scratch NULL, opts->workspace holds both (entmax_attn_workspace_size() bytes, the sum) and a
@@ -107,7 +111,11 @@ typedef struct {
  *   entmax_attn_fwd, bf16, d = 64, alpha <= 2:  to_f16_pass1, to_f16_pass2, fwd_h, mask_transpose
  *   entmax_attn_fwd, bf16, otherwise:           fwd_tc, mask_transpose
  *   entmax_attn_fwd, fp32:                      fwd_simt
- *   entmax_attn_bwd, d = 64, alpha <= 2:        to_f16_pass1, to_f16_pass2, bwd_pre, bwd_h_dq, bwd_h_dkdv
+ *   entmax_attn_bwd, d = 64, alpha <= 2:        to_f16_pass1, to_f16_pass2, bwd_pre, bwd_h_dq (keys of unit
+ *                                               scale), bwd_h_dq (delta pass, larger keys), bwd_h_dq (larger
+ *                                               keys), bwd_h_dkdv: of the three dQ launches, the range of K
+ *                                               lets either the first or the other two work; the rest return
+ *                                               at once
  *   entmax_attn_bwd, otherwise:                 bwd_pre, bwd_dkdv, bwd_dq
  *   softmax_attn_fwd, d = 64 with a workspace:  to_f16_pass1, to_f16_pass2, softmax_fwd_h
  *   softmax_attn_fwd, otherwise:                softmax_fwd
@@ -128,8 +136,9 @@ size_t entmax_attn_scratch_size(int B, int H, int n, int d, entmax_dtype dt, con
 
 /* Forward. Q, K, V: [B,H,n,d] inputs. O: [B,H,n,d] output (same dtype). tau: float32 [B,H,n]
  * output, the normaliser in z units. block_mask: uint32 output as described above. alpha > 1.
- * causal: 0 or 1. The workspace receives what the backward needs (sum_u, U V, the transposed mask and,
- * for bf16 with d = 64 and alpha <= 2, fp16 copies of Q, K, V with their range exponents).
+ * causal: 0 or 1. The workspace receives what the backward needs (sum_u, the transposed mask, U V for the
+ * bf16 and fp32 kernels and, for bf16 with d = 64 and alpha <= 2, fp16 copies of Q, K, V with their range
+ * exponents).
  * fp32 uses the FMA path. bf16 uses the tcgen05 path: with d = 64 and alpha <= 2 on fp16 operand copies
  * (exact for bf16 values of magnitude in [2^-14, 2^15), power-of-two scaled beyond), else on bf16
  * operands with two-term splits. */
@@ -188,8 +197,8 @@ entmax_status entmax_attn_selftest_timeout(int limit_us, void* stream);
 /* Human-readable name of a status code (static string). */
 const char* entmax_status_str(entmax_status s);
 
-/* Library ABI version: 2 (entmax_opts gained `events`, `num_events`, `scratch`, `scratch_bytes`; entmax_stats
- * gained `support`; entmax_attn_saved_size and entmax_attn_scratch_size were added). */
+/* Library ABI version: 2 (entmax_opts gained `events`, `num_events`, `scratch`, `scratch_bytes`, `alpha`;
+ * entmax_stats gained `support`; entmax_attn_saved_size and entmax_attn_scratch_size were added). */
 int entmax_attn_version(void);
 
 #ifdef __cplusplus

@@ -208,7 +208,8 @@ def test_separate_scratch_matches_single_buffer(torch_cuda, alpha, d):
         outs.append((f.O, f.tau, f.mask, dQ, dK, dV))
         if sep:
             Bsz, H, n, dd = t["Q"].shape
-            assert f.workspace.numel() == b.entmax_attn_saved_size(Bsz, H, n, dd)
+            assert f.workspace.numel() == b.entmax_attn_saved_size(Bsz, H, n, dd, b.ENTMAX_BF16,
+                                                                   b.make_opts(alpha=alpha))
     assert b.entmax_attn_check() == 0
     for name, x, y in zip(("O", "tau", "mask", "dQ", "dK", "dV"), *outs):
         assert torch_cuda.equal(x, y), name
