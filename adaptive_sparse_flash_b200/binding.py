@@ -39,6 +39,7 @@ EXPORTS = (
     "entmax_attn_fwd_noalloc",
     "entmax_attn_saved_size",
     "entmax_attn_scratch_size",
+    "softmax_attn_workspace_size",
 )
 
 
@@ -100,7 +101,8 @@ def lib() -> ctypes.CDLL:
     L = ctypes.CDLL(LIB_PATH)
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     op = ctypes.POINTER(EntmaxOpts)
-    for nm in ("entmax_attn_workspace_size", "entmax_attn_saved_size", "entmax_attn_scratch_size"):
+    for nm in ("entmax_attn_workspace_size", "entmax_attn_saved_size", "entmax_attn_scratch_size",
+               "softmax_attn_workspace_size"):
         getattr(L, nm).argtypes = [i, i, i, i, i, op]
         getattr(L, nm).restype = sz
     L.entmax_attn_fwd.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, f, i, i, op, vp]
@@ -195,11 +197,17 @@ def entmax_attn_scratch_size(B, H, n, d, dtype_code=ENTMAX_BF16, opts: EntmaxOpt
     return int(lib().entmax_attn_scratch_size(B, H, n, d, dtype_code, None if opts is None else ctypes.byref(opts)))
 
 
+def softmax_attn_workspace_size(B, H, n, d, dtype_code=ENTMAX_BF16, opts: EntmaxOpts | None = None) -> int:
+    return int(lib().softmax_attn_workspace_size(B, H, n, d, dtype_code,
+                                                  None if opts is None else ctypes.byref(opts)))
+
+
 def alloc_workspace(B, H, n, d, dtype_code=ENTMAX_BF16, device="cuda", opts=None, part="whole"):
-    """Device buffer for the workspace: part "whole" (saved + scratch in one buffer), "saved" or "scratch"."""
+    """Device buffer for the workspace: part "whole" (saved + scratch in one buffer), "saved" or "scratch";
+    "softmax" for the dense baseline's calls (no U V)."""
     import torch
     size_fn = {"whole": entmax_attn_workspace_size, "saved": entmax_attn_saved_size,
-               "scratch": entmax_attn_scratch_size}[part]
+               "scratch": entmax_attn_scratch_size, "softmax": softmax_attn_workspace_size}[part]
     nbytes = size_fn(B, H, n, d, dtype_code, opts)
     if nbytes == 0:
         raise EntmaxError(ENTMAX_ERR_INVALID, size_fn.__name__)
@@ -334,7 +342,7 @@ def softmax_forward(Q, K, V, causal=True, workspace=None, stream=None):
     O = torch.empty_like(Q)
     lse = torch.empty((B, H, n), dtype=torch.float32, device=Q.device)
     if workspace is None:
-        workspace = alloc_workspace(B, H, n, d, _dtype_code(Q), Q.device)
+        workspace = alloc_workspace(B, H, n, d, _dtype_code(Q), Q.device, part="softmax")
     opts = make_opts(workspace) if workspace is not False else None
     softmax_attn_fwd(Q, K, V, O, lse, causal, opts, stream)
     return O, lse
@@ -344,7 +352,7 @@ def softmax_backward(Q, K, V, O, lse, dO, causal=True, workspace=None, stream=No
     import torch
     B, H, n, d = Q.shape
     if workspace is None:
-        workspace = alloc_workspace(B, H, n, d, _dtype_code(Q), Q.device)
+        workspace = alloc_workspace(B, H, n, d, _dtype_code(Q), Q.device, part="softmax")
     opts = make_opts(workspace)
     dQ, dK, dV = (torch.empty(Q.shape, dtype=torch.float32, device=Q.device) for _ in range(3))
     softmax_attn_bwd(Q, K, V, O, dO, lse, dQ, dK, dV, causal, opts, stream)

@@ -92,6 +92,7 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 
 struct Dims {
     int B, H, n, d, mb, nqb, nkb, nw, nwq, bins, ntiles;
+    entmax_dtype dt;
 };
 
 entmax_status check_dims(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* o, Dims* out) {
@@ -108,7 +109,7 @@ entmax_status check_dims(int B, int H, int n, int d, entmax_dtype dt, const entm
     if (o && o->scale != 0.0f && !(o->scale > 0.0f && isfinite(o->scale))) return ENTMAX_ERR_INVALID;
     if (o && (o->num_events < 0 || (o->num_events > 0 && !o->events))) return ENTMAX_ERR_INVALID;
     Dims D;
-    D.B = B; D.H = H; D.n = n; D.d = d; D.mb = mb; D.bins = bins;
+    D.B = B; D.H = H; D.n = n; D.d = d; D.mb = mb; D.bins = bins; D.dt = dt;
     D.nqb = (n + mb - 1) / mb;
     D.nkb = (n + mb - 1) / mb;
     D.nw = (D.nkb + 31) / 32;
@@ -123,7 +124,8 @@ entmax_status check_dims(int B, int H, int n, int d, entmax_dtype dt, const entm
 //             bf16 and fp32 kernels (not the fp16 family, whose dQ kernel forms delta itself), U V (fp32
 //             [BH][n][d]);
 //   scratch - per call: delta and the row statistic padded to whole 64-row blocks ([BH][ceil(n/64)*64]) for
-//             the backward, the range words, and the fp16 operand copies of Q, K, V, dO (f16.cu).
+//             the backward, the range words, and (bf16 inputs with d = 64, the only shape an fp16 kernel
+//             serves) the fp16 operand copies of Q, K, V, dO (f16.cu).
 // With one buffer (opts->scratch NULL) the scratch part follows the saved part, and a backward reuses the
 // fp16 copies its forward left there; with a separate scratch buffer the backward makes its own copies.
 struct Workspace {
@@ -168,9 +170,10 @@ Workspace layout(const Dims& D, void* base, void* scratch, bool with_obar) {
     w.maxbits = reinterpret_cast<uint32_t*>(q + so);
     so = align256(so + 8 * sizeof(uint32_t));
     void** h16[4] = {&w.Qh, &w.Kh, &w.Vh, &w.dOh};
+    const bool with_h16 = D.dt == ENTMAX_BF16 && D.d == 64;
     for (int i = 0; i < 4; ++i) {
-        *h16[i] = q + so;
-        so = align256(so + rows * D.d * 2);
+        *h16[i] = with_h16 ? q + so : nullptr;
+        if (with_h16) so = align256(so + rows * D.d * 2);
     }
     w.scratch_bytes = so;
     return w;
@@ -228,7 +231,7 @@ using namespace eattn;
 
 extern "C" {
 
-EATTN_API int entmax_attn_version(void) { return 2; }
+EATTN_API int entmax_attn_version(void) { return 3; }
 
 EATTN_API const char* entmax_status_str(entmax_status s) {
     switch (s) {
@@ -260,6 +263,13 @@ EATTN_API size_t entmax_attn_scratch_size(int B, int H, int n, int d, entmax_dty
     Dims D;
     if (check_dims(B, H, n, d, dt, opts, &D) != ENTMAX_OK) return 0;
     return layout(D, nullptr, nullptr, false).scratch_bytes;
+}
+
+EATTN_API size_t softmax_attn_workspace_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts) {
+    Dims D;
+    if (check_dims(B, H, n, d, dt, opts, &D) != ENTMAX_OK) return 0;
+    const Workspace w = layout(D, nullptr, nullptr, false);
+    return w.saved_bytes + w.scratch_bytes;
 }
 
 EATTN_API entmax_status entmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* tau,

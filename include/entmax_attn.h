@@ -97,8 +97,8 @@ typedef struct {
  *             [B,H,n,d]); entmax_attn_saved_size() bytes. The size functions leave U V out only when
  *             opts->alpha names an alpha in (1, 2] (with d = 64, bf16); a workspace sized without U V
  *             makes calls with another alpha return ENTMAX_ERR_WORKSPACE;
- *   scratch - used within one call: the fp16 operand copies of Q, K, V, dO, the padded per-row delta and
- *             row statistic, range words; entmax_attn_scratch_size() bytes.
+ *   scratch - used within one call: the padded per-row delta and row statistic, range words and, for bf16
+ *             inputs with d = 64, the fp16 operand copies of Q, K, V, dO; entmax_attn_scratch_size() bytes.
  * With opts->scratch NULL, opts->workspace holds both (entmax_attn_workspace_size() bytes, the sum) and a
  * backward reuses the fp16 copies of Q, K, V that its forward left there. With opts->scratch set,
  * opts->workspace needs only the saved part: only that must be kept from the forward to the backward (the
@@ -163,10 +163,14 @@ entmax_status entmax_attn_bwd(const void* Q, const void* K, const void* V, const
 entmax_status softmax_attn_fwd(const void* Q, const void* K, const void* V, void* O, float* lse,
                                int B, int H, int n, int d, int causal, entmax_dtype dt,
                                const entmax_opts* opts, void* stream);
-/* softmax_attn_bwd: dQ, dK, dV float32 like entmax_attn_bwd; needs opts->workspace (same size query). */
+/* softmax_attn_bwd: dQ, dK, dV float32 like entmax_attn_bwd; needs opts->workspace
+ * (softmax_attn_workspace_size() bytes, or any entmax size for the same shape). */
 entmax_status softmax_attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                                const float* lse, void* dQ, void* dK, void* dV, int B, int H, int n, int d,
                                int causal, entmax_dtype dt, const entmax_opts* opts, void* stream);
+/* Bytes of workspace (one buffer) that softmax_attn_fwd/bwd need: the entmax layout without U V
+ * (the dense baseline keeps no U V). 0 for invalid sizes. opts may be NULL. */
+size_t softmax_attn_workspace_size(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* opts);
 
 /* Forward that allocates nothing and needs no workspace (the paper has no counterpart: this is for
  * callers that cannot allocate device memory, e.g. code running inside a framework that owns the whole
@@ -197,8 +201,10 @@ entmax_status entmax_attn_selftest_timeout(int limit_us, void* stream);
 /* Human-readable name of a status code (static string). */
 const char* entmax_status_str(entmax_status s);
 
-/* Library ABI version: 2 (entmax_opts gained `events`, `num_events`, `scratch`, `scratch_bytes`, `alpha`;
- * entmax_stats gained `support`; entmax_attn_saved_size and entmax_attn_scratch_size were added). */
+/* Library ABI version: 3. Version 2: entmax_opts gained `events`, `num_events`, `scratch`, `scratch_bytes`,
+ * `alpha`; entmax_stats gained `support`; entmax_attn_saved_size and entmax_attn_scratch_size were added.
+ * Version 3: softmax_attn_workspace_size was added; the scratch part holds fp16 operand copies only for
+ * bf16 inputs with d = 64. */
 int entmax_attn_version(void);
 
 #ifdef __cplusplus

@@ -37,7 +37,7 @@ def test_library_exports_every_symbol(L):
 
 def test_version_and_status_strings(L):
     from adaptive_sparse_flash_b200 import binding as b
-    assert L.entmax_attn_version() == 2
+    assert L.entmax_attn_version() == 3
     for s in range(7):
         assert len(b.entmax_status_str(s)) > 0
     assert b.entmax_status_str(99) == "unknown status"
@@ -53,6 +53,35 @@ def test_workspace_size(L):
     assert b.entmax_attn_workspace_size(1, 16, n, 96) == 0     # d unsupported
     assert b.entmax_attn_workspace_size(0, 16, n, 64) == 0     # empty batch
     assert b.entmax_attn_workspace_size(1, 1, 0, 64) == 0      # empty sequence
+
+
+def _a256(x):
+    return (x + 255) // 256 * 256
+
+
+@pytest.mark.parametrize("B,H,n,d,dt,alpha,with_uv,with_h16", [
+    (1, 16, 16384, 64, 0, 1.5, False, True),   # fp16 kernels: no U V, fp16 copies in the scratch
+    (1, 16, 16384, 64, 0, 3.0, True, True),    # alpha > 2: bf16 kernels keep U V
+    (1, 16, 16384, 64, 0, 0.0, True, True),    # alpha unknown: sized for any alpha
+    (2, 16, 4096, 128, 0, 1.5, True, False),   # d = 128: bf16 kernels, no fp16 copies
+    (1, 1, 256, 64, 1, 1.5, True, False),      # fp32 inputs: FMA kernel, no fp16 copies
+    (3, 5, 1000, 64, 0, 2.0, False, True),     # ragged n
+])
+def test_workspace_parts(L, B, H, n, d, dt, alpha, with_uv, with_h16):
+    """The saved and scratch parts hold exactly the buffers the header lists for the call's kernels."""
+    from adaptive_sparse_flash_b200 import binding as b
+    o = b.make_opts(alpha=alpha)
+    o.mask_block = 32 if dt == 1 else 0
+    mb = 32 if dt == 1 else 64
+    rows, nb = B * H * n, (n + mb - 1) // mb
+    rows_pad = B * H * ((n + 63) // 64) * 64
+    saved = (_a256(rows * d * 4) if with_uv else 0) + _a256(rows * 4) + _a256(B * H * nb * ((nb + 31) // 32) * 4)
+    scratch = 2 * _a256(rows_pad * 4) + _a256(8 * 4) + (4 * _a256(rows * d * 2) if with_h16 else 0)
+    assert b.entmax_attn_saved_size(B, H, n, d, dt, o) == saved
+    assert b.entmax_attn_scratch_size(B, H, n, d, dt, o) == scratch
+    assert b.entmax_attn_workspace_size(B, H, n, d, dt, o) == saved + scratch
+    saved_sm = saved - (_a256(rows * d * 4) if with_uv else 0)  # the dense baseline keeps no U V
+    assert b.softmax_attn_workspace_size(B, H, n, d, dt, o) == saved_sm + scratch
 
 
 def _fwd(L, ptr=16, n=64, d=64, alpha=1.5, causal=1, dt=0, ws=True, mask_block=0, bins=0, init_mode=0,
