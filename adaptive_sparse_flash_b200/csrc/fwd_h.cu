@@ -6,10 +6,14 @@
 //                   and reads TMEM lane r; the two warpgroups take alternate key blocks of every sweep;
 //   warp 8          S issue (one thread): S = Q K^T from shared memory into three TMEM buffers per
 //                   warpgroup;
-//   warp 10         P V issue (one thread): O += P V with P stored by the compute warps into the TMEM
-//                   columns of the S tile it came from. Two issuing threads keep the tensor pipe fed: each
-//                   waits only on its own barriers, in block order;
+//   warp 10         P V issue (one thread): O_g += P V with P stored by the compute warps into the TMEM
+//                   columns of the S tile it came from, into one accumulator per warpgroup (consecutive
+//                   products then never feed one another). Two issuing threads keep the tensor pipe fed:
+//                   each waits only on its own barriers, in block order;
 //   warp 9          TMA issue (one thread): Q once, K blocks of 64 keys and, in P V sweeps, V blocks.
+// A K ring slot is released by the four warps that read the S tile it fed (once they see that S tile
+// complete, the MMA that read the slot has completed too), so that the S thread commits once per tile:
+// each tcgen05.commit costs the issuing thread tens of cycles.
 //
 // P lies in [0, 1] for alpha <= 2 and enters P V as one fp16 term (11 significant bits; bf16 would need a
 // two-term split). The backward needs no product of u with V from the forward: its dQ kernel forms
@@ -20,7 +24,8 @@
 // alone.
 //
 // TMEM columns (512): S buffer b (of three) of warpgroup g at 64 (3 g + b), holding P in its first 32
-// columns (K step kk of 16 keys is columns 8 kk .. 8 kk + 7) in P V sweeps; O at 384.
+// columns (K step kk of 16 keys is columns 8 kk .. 8 kk + 7) in P V sweeps; O_0 at 384, O_1 at 448 (their
+// sum is O).
 //
 // Sweeps follow the plan protocol of the bf16 forward (fwd_tc.cu): before each sweep the compute warps
 // publish its kind and its set of key blocks, which the issuing warps follow.
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         mbar_init(&sm.q_full, 1);
-        for (int i = 0; i < NKS; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 1); }
+        for (int i = 0; i < NKS; ++i) { mbar_init(&sm.k_full[i], 1); mbar_init(&sm.k_empty[i], 4); }
         for (int i = 0; i < NVS; ++i) { mbar_init(&sm.v_full[i], 1); mbar_init(&sm.v_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
             for (int b = 0; b < NSB; ++b) {
@@ -365,7 +370,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int kk = 0; kk < D / 16; ++kk)
                         mma_ss(dS, sdesc_at(kDescK, sQ + kk * 32), sdesc_at(kDescK, kbase + kk * 32), idS, kk > 0 ? 1u : 0u);
                     mma_commit(&sm.s_full[g][b]);
-                    mma_commit(&sm.k_empty[ks]);
                     ++lc;
                     if (g) ++sc1; else ++sc0;
                 }
@@ -413,8 +417,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int kk = 0; kk < BN / 16; ++kk) {
                         const uint64_t dv = sdesc_at(kDescMN, vbase + kk * 2048);
-                        const uint32_t acc = (tp == 0 && kk == 0) ? 0u : 1u;
-                        mma_ts(tmem + kColO, tpu + 8 * kk, dv, idPV, acc);
+                        const uint32_t acc = (tp == g && kk == 0) ? 0u : 1u;
+                        mma_ts(tmem + kColO + 64u * g, tpu + 8 * kk, dv, idPV, acc);
                     }
                     mma_commit(&sm.pv_free[g][b]);
                     mma_commit(&sm.v_empty[vs]);
@@ -470,7 +474,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         float vbuf[BN];
 
-        auto load_S = [&]() -> bool {
+        uint32_t lcs = 0;  // K blocks of the sweeps before this one (ring order)
+        auto load_S = [&](uint32_t kidx) -> bool {
             const uint32_t sb = sc % NSB;
             const bool got = wait_bounded(&sm.s_full[g][sb], (sc / NSB) & 1, abort_flag, a.status);
             if (!__all_sync(0xffffffffu, got)) return false;
@@ -484,7 +489,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.s_empty[g][sb]);
+            if (lane == 0) {
+                mbar_arrive(&sm.s_empty[g][sb]);
+                mbar_arrive(&sm.k_empty[kidx % NKS]);  // the MMA that read this K block has completed
+            }
             ++sc;
             return true;
         };
@@ -530,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ovf = false;
         volatile float* xm_other = sm.xf[kXMax0 + (g ^ 1)];
         for (int J = g; J < nblk && ok; J += 2) {
-            if (!(ok = load_S())) break;
+            if (!(ok = load_S(lcs + J))) break;
             mask_S(J);
             const float amax = group_max();
             // the other warpgroup's running max is a valid (tighter) threshold as well
@@ -567,6 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t ball = __ballot_sync(0xffffffffu, any);
             if (lane == 0 && ball) atomicOr(&next[J >> 5], 1u << (J & 31));
         }
+        lcs += nblk;
         if (g == 1) sm.xf[kXCnt1][r] = __int_as_float(ovf ? -1 : nst);
         ok = !bar_or256(!ok || *abort_flag != 0);
 
@@ -621,12 +630,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (mine) hist_start(h, m_raw, sp);
                 const float thr_f = m_raw - sp.inv_cz;
                 const uint32_t* bits_p = plan_bits + (sw & 1) * W;
+                uint32_t ph = 0;
                 for (int wd = 0; wd < W && ok; ++wd) {
                     uint32_t bits = bits_p[wd];
                     while (bits) {
                         const int J = wd * 32 + __ffs(bits) - 1;
                         bits &= bits - 1;
-                        if (!(ok = load_S())) break;
+                        if (!(ok = load_S(lcs + ph++))) break;  // warpgroup 0 takes every block
                         mask_S(J);
                         const float amax = group_max();
                         const bool keep = amax > thr_f;
@@ -647,6 +657,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (lane == 0 && ball) atomicOr(&next[J >> 5], 1u << (J & 31));
                     }
                 }
+            }
+            {
+                const uint32_t* bp = plan_bits + (sw & 1) * W;
+                for (int wd = 0; wd < W; ++wd) lcs += __popc(bp[wd]);
             }
             ok = !bar_or256(!ok || *abort_flag != 0);
             if (ok && g == 0 && valid && row_ovf) {
@@ -679,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int J = wd * 32 + __ffs(bits) - 1;
                     bits &= bits - 1;
                     if (((p++) & 1) != g) continue;
-                    if (!(ok = load_S())) break;
+                    if (!(ok = load_S(lcs + (uint32_t)(p - 1)))) break;
                     mask_S(J);
                     const float amax = group_max();
                     const bool keep = sp.cz * amax > lo0;
@@ -729,11 +743,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 solve_step(s, F0, F1, F2, F0b, sp);
                 last_step = s.tau - before;
             }
+            lcs += (uint32_t)p;
             ++refine;
         };
 
         // ---- P V sweep: p to TMEM for the P V MMAs, exact mask, sum check ----
         float Su = 0.f;
+        int pv_tiles = 0;  // blocks of the last P V sweep
         auto pv_sweep = [&]() -> bool {
             if (g == 0) {
                 sm.xf[kXTau][r] = s.tau;
@@ -752,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int J = wd * 32 + __ffs(bits) - 1;
                     bits &= bits - 1;
                     if (((p++) & 1) != g) continue;
-                    if (!(ok = load_S())) break;
+                    if (!(ok = load_S(lcs + (uint32_t)(p - 1)))) break;
                     mask_S(J);
                     const float amax = group_max();
                     const bool keep = sp.cz * amax > lo0;
@@ -827,6 +843,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 sm.xf[kXF2][r] = F2;
                 sm.xf[kXCnt][r] = __uint_as_float(Sn);
             }
+            pv_tiles = p;
+            lcs += (uint32_t)p;
             ++pv;
             ok = !bar_or256(!ok || *abort_flag != 0);
             bool changed = false;
@@ -869,6 +887,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t o[32];
             tmem_ld32(lane_base + kColO + 32u * g, o);
             tmem_ld_wait();
+            if (pv_tiles > 1) {  // the second warpgroup's accumulator holds the odd blocks
+                uint32_t o2[32];
+                tmem_ld32(lane_base + kColO + 64u + 32u * g, o2);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) + __uint_as_float(o2[i]));
+            }
             if (valid) {
                 uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + (head + row) * D + 32 * g);
 #pragma unroll

@@ -14,7 +14,8 @@
 //   O = (2^(m_0 - m) O_0 + 2^(m_1 - m) O_1) / (2^(m_0 - m) l_0 + 2^(m_1 - m) l_1),  m = max(m_0, m_1),
 //   lse = ln 2 (m + log2 l).
 // TMEM columns: S buffer b of warpgroup g at 64 (2 g + b) (P in its first 32), O_g at 256 + 64 g.
-// A new S tile enters a buffer only after the P V product that read its P completed.
+// A new S tile enters a buffer only after the P V product that read its P completed. A K ring slot is
+// released by the four warps that read the S tile it fed (one commit per tile in the S thread).
 // ("faster than FlashAttention-2 above ~60% block sparsity": AdaSplash-2, gist.science (de), section 4.)
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -100,7 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         mbar_init(&bb.q_full, 1);
-        for (int i = 0; i < NKS; ++i) { mbar_init(&bb.k_full[i], 1); mbar_init(&bb.k_empty[i], 1); }
+        for (int i = 0; i < NKS; ++i) { mbar_init(&bb.k_full[i], 1); mbar_init(&bb.k_empty[i], 4); }
         for (int i = 0; i < NVS; ++i) { mbar_init(&bb.v_full[i], 1); mbar_init(&bb.v_empty[i], 1); }
         for (int g = 0; g < 2; ++g)
             for (int b = 0; b < 2; ++b) {
@@ -175,7 +176,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mma_ss(tmem + 64u * bi, sdesc_at(kDescK, sQ + kk * 32), sdesc_at(kDescK, kbase + kk * 32), idS,
                            kk > 0 ? 1u : 0u);
                 mma_commit(&bb.s_full[g][b]);
-                mma_commit(&bb.k_empty[ks]);
             }
             mma_commit(&bb.drain[0]);
             wait_drain(&bb.drain[0], 0, 200000000ull);
@@ -230,7 +230,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bb.s_empty[g][b]);
+            if (lane == 0) {
+                mbar_arrive(&bb.s_empty[g][b]);
+                mbar_arrive(&bb.k_empty[(uint32_t)t % NKS]);  // the MMA that read K block t has completed
+            }
             const int k0 = t * BN;
             const bool full = valid && k0 + BN <= a.n && (!a.causal || k0 + BN - 1 <= row0);
             if (__any_sync(0xffffffffu, !full)) {
