@@ -291,15 +291,17 @@ __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, cons
                 const int jn = (stop - sl) & (B - 1);  // offset of this bin below the top
                 const int J1 = jn + 1;                 // first J at which the bin counts
                 if (A0 > 0) {
-                    const long long t = first_cross();
-                    if (J0 + t < J1) {  // crosses before this bin starts to count
+                    const long long T = J1 - J0;
+                    // crosses before this bin starts to count iff A_k(J1 - 1) reaches thr (A_k is
+                    // nondecreasing in J); only then is the crossing located
+                    if (T >= 2 && Ak(T - 1) >= thr) {
+                        const long long t = first_cross();
                         A2 = (KIND == kAlpha15) ? Ak(t) : A2;
                         A1 += t * A0;
                         J = J0 + (int)t;
                         found = true;
                         break;
                     }
-                    const long long T = J1 - J0;
                     A2 += 2 * T * A1 + T * T * A0;
                     A1 += T * A0;
                 }
