@@ -98,6 +98,8 @@ struct Dims {
 entmax_status check_dims(int B, int H, int n, int d, entmax_dtype dt, const entmax_opts* o, Dims* out) {
     if (B < 1 || H < 1 || n < 1 || d < 1) return ENTMAX_ERR_INVALID;
     if ((long long)B * H > (1ll << 30) || (long long)n > (1ll << 30)) return ENTMAX_ERR_INVALID;
+    // the kernels' grids are (B*H, tiles of 128 rows); a grid's y extent is at most 65535
+    if ((long long)n > 65535ll * kTileRows) return ENTMAX_ERR_UNSUPPORTED;
     if (dt != ENTMAX_BF16 && dt != ENTMAX_FP32) return ENTMAX_ERR_INVALID;
     if (d != 64 && d != 128) return ENTMAX_ERR_UNSUPPORTED;
     const int mb = (o && o->mask_block) ? o->mask_block : 64;

@@ -191,8 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* vis = reinterpret_cast<uint32_t*>(&bb + 1);  // [nwq] query blocks to visit
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int kt = blockIdx.x;
-    const int bh = blockIdx.y;
+    const int kt = blockIdx.y;  // grid (B*H, key tiles): the longest (first) key tiles of every head first
+    const int bh = blockIdx.x;
     const int k0 = kt * TM;
     const int nwq = a.nwq;
     const int npad = a.nqb * TB;
@@ -497,8 +497,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* vis = reinterpret_cast<uint32_t*>(&bb + 1);  // [nw] key blocks to visit
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qt = (int)gridDim.x - 1 - (int)blockIdx.x;
-    const int bh = blockIdx.y;
+    const int qt = (int)gridDim.y - 1 - (int)blockIdx.y;  // grid (B*H, tiles): longest tiles of every head first
+    const int bh = blockIdx.x;
     const int q0 = qt * TM;
     const int nw = a.nw;
     const int npad = a.nqb * TB;
@@ -759,7 +759,7 @@ cudaError_t launch_t(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaSt
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
             return e;
         launch_mark(stream);
-        kern<<<dim3(ntiles, BH), kThreads, bytes, stream>>>(tq64, tk128, tv128, tdo64, a, delta_pad, stat_pad);
+        kern<<<dim3(BH, ntiles), kThreads, bytes, stream>>>(tq64, tk128, tv128, tdo64, a, delta_pad, stat_pad);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
@@ -769,7 +769,7 @@ cudaError_t launch_t(const BwdArgs& a, float* delta_pad, float* stat_pad, cudaSt
         if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
             return e;
         launch_mark(stream);
-        kern<<<dim3(ntiles, BH), kThreads, bytes, stream>>>(tq128, tk64, tv64, tdo128, a, delta_pad, stat_pad);
+        kern<<<dim3(BH, ntiles), kThreads, bytes, stream>>>(tq128, tk64, tv64, tdo128, a, delta_pad, stat_pad);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;

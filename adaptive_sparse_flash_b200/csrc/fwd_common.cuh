@@ -34,7 +34,7 @@ struct FwdArgs {
     const uint32_t* maxbits;  // [3]: Q, K, V
 };
 
-enum SweepKind : int { kSweepDense = 0, kSweepRefine = 1, kSweepPV = 2, kSweepDone = 3, kSweepHist = 4 };
+enum SweepKind : int { kSweepDense = 0, kSweepRefine = 1, kSweepPV = 2, kSweepDone = 3, kSweepHist = 4, kSweepSupport = 5 };
 
 // Number of allowed keys of query row `row`.
 __device__ __forceinline__ int allowed_keys(int row, int n, int causal) {

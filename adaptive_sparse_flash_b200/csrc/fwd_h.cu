@@ -36,7 +36,12 @@
 //             bins those rows' entries into their histograms with the window fixed by the final max;
 //   refine  - candidate blocks: solver sums at the current tau (partial sums of the two warpgroups are
 //             combined by warpgroup 0, which owns the solver state of each row);
-//   P V     - candidate blocks: p to TMEM for the P V MMAs, exact block mask, sum check.
+//   P V     - candidate blocks: p to TMEM for the P V MMAs, exact block mask, sum check;
+//   support - instead of P V, when every row of the tile was solved on chip from its stash and has at most
+//             kElemCap support entries per warpgroup: candidate blocks, S recomputed only to find the
+//             support (exact block mask); each warpgroup lists the (key, p) of its blocks' support entries
+//             in shared memory, and O = sum p v is then gathered from those rows of V in fp32 (element
+//             sparsity: no P V MMAs and no V ring).
 // (AdaSplash-2, gist.science (de), section 2: histogram initialisation, hybrid solver, bit-packed block
 // mask, only nonzero blocks processed.)
 #include <cuda.h>
@@ -89,6 +94,12 @@ struct HCfg {
     static constexpr uint32_t offSmall = offStash + kStashBytes;
     static constexpr int kStride = NB == 512 ? kLiveStride512 : kLiveStride;  // live words per row + 1
     static_assert(NVS * kKBytes <= kHistBytes, "V ring must fit the histogram region");
+    // element path: per row and warpgroup a list of up to kElemCap support entries (key u16, p f32) and its
+    // length, in the histogram region once tau is solved
+    static constexpr int kElemCap = 40;
+    static constexpr uint32_t kElemKeys = 2u * kElemCap * BM * 2u;
+    static constexpr uint32_t kElemP = 2u * kElemCap * BM * 4u;
+    static_assert(kElemKeys + kElemP + 2u * BM * 4u <= kHistBytes, "support lists must fit the histogram region");
 };
 
 constexpr uint32_t kTmemCols = 512;
@@ -235,13 +246,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* mrow = next + W;                                   // [2][W]
     uint32_t* live_all = mrow + 2 * W;                           // [128][HC::kStride]
     uint16_t* hist = reinterpret_cast<uint16_t*>(smem + offHist);
+    uint16_t* elem_key = reinterpret_cast<uint16_t*>(smem + offHist);                        // [2][cap][128]
+    float* elem_p = reinterpret_cast<float*>(smem + offHist + HC::kElemKeys);                   // [2][cap][128]
+    int* elem_cnt = reinterpret_cast<int*>(smem + offHist + HC::kElemKeys + HC::kElemP);        // [2][128]
     float* stash = reinterpret_cast<float*>(smem + offStash);
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int qt = a.ntiles - 1 - (int)blockIdx.x;
-    const int bh = blockIdx.y;
+    // grid (B*H, tiles): the longest causal tiles of every head first
+    const int qt = a.ntiles - 1 - (int)blockIdx.y;
+    const int bh = blockIdx.x;
     const int row0 = qt * BM;
     const int kend = a.causal ? min(a.n, row0 + BM) : a.n;
     const int nblk = (kend + BN - 1) / BN;
@@ -514,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 plan_bits[nb * W + i] = next[i];
                 next[i] = 0u;
             }
-            if (kind == kSweepPV)
+            if (kind == kSweepPV || kind == kSweepSupport)
                 for (int i = tid; i < 2 * W; i += kCompute) mrow[i] = 0u;
             if (tid == 0) sm.plan_kind[nb] = kind;
             named_bar_sync(1, kCompute);
@@ -872,22 +887,116 @@ __global__ void __launch_bounds__(kThreads, 1)
                 refine_sweep();
             } while (ok && refine < kMaxSweeps && bar_or256(g == 0 && !s.done && fabsf(last_step) > sp.w));
         }
-        while (ok) {
-            const bool changed = pv_sweep();
-            if (!ok || !changed || pv >= 3) break;
-            while (ok && refine < kMaxSweeps && bar_or256(g == 0 && !s.done)) refine_sweep();
+        // ---- support sweep (element path): list the support entries of each row, then gather O ----
+        constexpr int kCap = HC::kElemCap;
+        float oacc[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) oacc[i] = 0.f;
+        auto support_sweep = [&]() {
+            if (g == 0) sm.xf[kXTau][r] = s.tau;
+            publish(kSweepSupport);
+            const float t = sm.xf[kXTau][r];
+            uint16_t* lk = elem_key + g * (kCap * BM) + r;
+            float* lp = elem_p + g * (kCap * BM) + r;
+            int cnt = 0;
+            const uint32_t* bits_p = plan_bits + (sw & 1) * W;
+            int p = 0;
+            for (int wd = 0; wd < W && ok; ++wd) {
+                uint32_t bits = bits_p[wd];
+                while (bits) {
+                    const int J = wd * 32 + __ffs(bits) - 1;
+                    bits &= bits - 1;
+                    if (((p++) & 1) != g) continue;
+                    if (!(ok = load_S(lcs + (uint32_t)(p - 1)))) break;
+                    mask_S(J);
+                    const float amax = group_max();
+                    const bool nz = fmaf(amax, sp.cz, -t) > 0.f;
+                    if (nz) {
+                        // the row's support entries in this block (groups of 8 whose max is above tau); the
+                        // same S and the same x as the solver's count, so the list never exceeds the row's
+                        // support (the cap check only guards the memory)
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            if (fmaf(gm[q], sp.cz, -t) > 0.f) {
+#pragma unroll
+                                for (int e = 0; e < 8; ++e) {
+                                    const float x = fmaf(vbuf[8 * q + e], sp.cz, -t);
+                                    if (x > 0.f && cnt < kCap) {
+                                        lk[cnt * BM] = (uint16_t)(J * BN + 8 * q + e);
+                                        lp[cnt * BM] = pow_k<KIND>(x, sp.k);
+                                        ++cnt;
+                                    }
+                                }
+                            }
+                        }
+                    }
+                    const uint32_t nb = __ballot_sync(0xffffffffu, nz);
+                    if (lane == 0 && nb) atomicOr(&mrow[half * W + (J >> 5)], 1u << (J & 31));
+                }
+            }
+            lcs += (uint32_t)p;
+            elem_cnt[g * BM + r] = cnt;
+            ++pv;
+            ok = !bar_or256(!ok || *abort_flag != 0);  // lists and counts of both warpgroups visible
+            if (g == 0) Su = Su_stash;
+            // O row r, columns 32 g .. 32 g + 31: sum over both lists of p v_key (fp16 copy of V, fp32 sums)
+            if (ok && valid) {
+                const __half* Vh = static_cast<const __half*>(a.Vh) + head * D + 32 * g;
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int nh = elem_cnt[hh * BM + r];
+                    const uint16_t* kk = elem_key + hh * (kCap * BM) + r;
+                    const float* pk = elem_p + hh * (kCap * BM) + r;
+#pragma unroll 2
+                    for (int e = 0; e < nh; ++e) {
+                        const uint4* src = reinterpret_cast<const uint4*>(Vh + (size_t)kk[e * BM] * D);
+                        const float pe = pk[e * BM];
+                        uint4 w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) w[i] = __ldg(src + i);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const __half2* h2 = reinterpret_cast<const __half2*>(&w[i]);
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) {
+                                const float2 f = __half22float2(h2[m]);
+                                oacc[8 * i + 2 * m] = fmaf(pe, f.x, oacc[8 * i + 2 * m]);
+                                oacc[8 * i + 2 * m + 1] = fmaf(pe, f.y, oacc[8 * i + 2 * m + 1]);
+                            }
+                        }
+                    }
+                }
+            }
+        };
+
+        // element path: no row overflowed its stash, every row's tau is final, every support fits a list
+        // (and keys fit the u16 lists)
+        const bool elem = ok && a.n <= 65536 &&
+                          !bar_or256(g == 0 && valid && !(!row_ovf && s.done && nsup <= (uint32_t)kCap));
+        if (elem) {
+            support_sweep();
+        } else {
+            while (ok) {
+                const bool changed = pv_sweep();
+                if (!ok || !changed || pv >= 3) break;
+                while (ok && refine < kMaxSweeps && bar_or256(g == 0 && !s.done)) refine_sweep();
+            }
         }
 
         // ---- wait for the last P V MMAs, then write O (warpgroup g: columns 32 g .. 32 g + 31), tau, sum u ----
-        if (ok) ok = __all_sync(0xffffffffu, wait_bounded(&sm.o_full, (pv - 1) & 1, abort_flag, a.status));
+        if (ok && !elem) ok = __all_sync(0xffffffffu, wait_bounded(&sm.o_full, (pv - 1) & 1, abort_flag, a.status));
         ok = !bar_or256(!ok || *abort_flag != 0);
         if (ok) {
             tc_fence_after();
             __syncwarp();
             uint32_t o[32];
-            tmem_ld32(lane_base + kColO + 32u * g, o);
-            tmem_ld_wait();
-            if (pv_tiles > 1) {  // the second warpgroup's accumulator holds the odd blocks
+            if (elem) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(oacc[i]);
+            } else {
+                tmem_ld32(lane_base + kColO + 32u * g, o);
+                tmem_ld_wait();
+            }
+            if (!elem && pv_tiles > 1) {  // the second warpgroup's accumulator holds the odd blocks
                 uint32_t o2[32];
                 tmem_ld32(lane_base + kColO + 64u + 32u * g, o2);
                 tmem_ld_wait();
@@ -967,7 +1076,7 @@ cudaError_t launch_fwd_h_t(const FwdArgs& a, cudaStream_t stream) {
     auto kern = fwd_h_kernel<KIND, NB>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
         return e;
-    dim3 grid(a.ntiles, a.B * a.H);
+    dim3 grid(a.B * a.H, a.ntiles);
     launch_mark(stream);
     kern<<<grid, kThreads, bytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError();

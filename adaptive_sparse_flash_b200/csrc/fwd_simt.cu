@@ -79,8 +79,8 @@ __global__ void __launch_bounds__(128, 1) fwd_simt_kernel(const FwdArgs a) {
     __shared__ TileStats st;
 
     const int tid = threadIdx.x;
-    const int qt = a.ntiles - 1 - (int)blockIdx.x;
-    const int bh = blockIdx.y;
+    const int qt = a.ntiles - 1 - (int)blockIdx.y;  // grid (B*H, tiles): longest tiles of every head first
+    const int bh = blockIdx.x;
     const int row = qt * kTileRows + tid;
     const bool valid = row < a.n;
     const int n_i = valid ? allowed_keys(row, a.n, a.causal) : 1;
@@ -316,7 +316,7 @@ cudaError_t launch_t(const FwdArgs& a, cudaStream_t stream) {
     auto kern = fwd_simt_kernel<T, D, KIND>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
     if (e != cudaSuccess) return e;
-    dim3 grid(a.ntiles, a.B * a.H);
+    dim3 grid(a.B * a.H, a.ntiles);
     launch_mark(stream);
     kern<<<grid, 128, bytes, stream>>>(a);
     return cudaGetLastError();

@@ -163,8 +163,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int qt = a.ntiles - 1 - (int)blockIdx.x;
-    const int bh = blockIdx.y;
+    const int qt = a.ntiles - 1 - (int)blockIdx.y;  // grid (B*H, tiles): longest tiles of every head first
+    const int bh = blockIdx.x;
     const int row0 = qt * BM;
     const int kend = a.causal ? min(a.n, row0 + BM) : a.n;
     const int nblk = (kend + BN - 1) / BN;
@@ -806,7 +806,7 @@ static cudaError_t launch_fwd_tc_t(const FwdArgs& a, cudaStream_t stream) {
     auto kern = fwd_tc_kernel<D, KIND>;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
         return e;
-    dim3 grid(a.ntiles, a.B * a.H);
+    dim3 grid(a.B * a.H, a.ntiles);
     launch_mark(stream);
     kern<<<grid, kThreads, bytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError();

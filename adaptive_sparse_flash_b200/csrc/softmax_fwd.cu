@@ -59,8 +59,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char* smem = align_smem_1024(smem_raw);
     BarsS& bb = *reinterpret_cast<BarsS*>(smem + C::offBar);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qt = a.ntiles - 1 - (int)blockIdx.x;
-    const int bh = blockIdx.y;
+    const int qt = a.ntiles - 1 - (int)blockIdx.y;  // grid (B*H, tiles): longest tiles of every head first
+    const int bh = blockIdx.x;
     const int row0 = qt * BM;
     const int kend = a.causal ? min(a.n, row0 + BM) : a.n;
     const int nblk = (kend + BN - 1) / BN;
@@ -281,7 +281,7 @@ cudaError_t launch_t(const SoftmaxFwdArgs& a, cudaStream_t stream) {
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) != cudaSuccess)
         return e;
     launch_mark(stream);
-    kern<<<dim3(a.ntiles, BH), kThreads, bytes, stream>>>(tq, tk, tv, a);
+    kern<<<dim3(BH, a.ntiles), kThreads, bytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError();
 }
 

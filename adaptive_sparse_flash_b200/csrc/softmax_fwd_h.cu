@@ -92,8 +92,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* xl = xm + BM;                                 // [128]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int qt = a.ntiles - 1 - (int)blockIdx.x;
-    const int bh = blockIdx.y;
+    const int qt = a.ntiles - 1 - (int)blockIdx.y;  // grid (B*H, tiles): longest tiles of every head first
+    const int bh = blockIdx.x;
     const int row0 = qt * BM;
     const int kend = a.causal ? min(a.n, row0 + BM) : a.n;
     const int T = (kend + BN - 1) / BN;  // key blocks of this tile
@@ -354,7 +354,7 @@ cudaError_t launch_softmax_fwd_h(const SoftmaxFwdArgs& a, cudaStream_t stream) {
     if ((e = cudaFuncSetAttribute(softmax_fwd_h_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes)) !=
         cudaSuccess)
         return e;
-    dim3 grid(a.ntiles, a.B * a.H);
+    dim3 grid(a.B * a.H, a.ntiles);
     launch_mark(stream);
     softmax_fwd_h_kernel<<<grid, kThreads, bytes, stream>>>(tq, tk, tv, a);
     return cudaGetLastError();

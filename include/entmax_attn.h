@@ -47,7 +47,8 @@ extern "C" {
 typedef enum {
     ENTMAX_OK = 0,
     ENTMAX_ERR_INVALID = 1,     /* null pointer, bad size, alpha <= 1, workspace too small for ... */
-    ENTMAX_ERR_UNSUPPORTED = 2, /* valid but not built: d not in {64, 128}, fp32 backward, ...     */
+    ENTMAX_ERR_UNSUPPORTED = 2, /* valid but not built: d not in {64, 128}, fp32 backward,
+                                   n > 65535 * 128, ...                                         */
     ENTMAX_ERR_ALIGN = 3,       /* a tensor base address is not 16-byte aligned                    */
     ENTMAX_ERR_CUDA = 4,        /* a CUDA runtime / driver call failed                             */
     ENTMAX_ERR_TIMEOUT = 5,     /* a device-side bounded wait ran out (reported by check())        */

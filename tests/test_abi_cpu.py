@@ -108,6 +108,7 @@ def test_validation_errors_return_before_launch(L):
     assert _fwd(L, causal=2) == b.ENTMAX_ERR_INVALID
     assert _fwd(L, n=0) == b.ENTMAX_ERR_INVALID
     assert _fwd(L, d=80) == b.ENTMAX_ERR_UNSUPPORTED
+    assert _fwd(L, n=65535 * 128 + 1) == b.ENTMAX_ERR_UNSUPPORTED  # beyond the grid's tile extent
     assert _fwd(L, dt=7) == b.ENTMAX_ERR_INVALID
     assert _fwd(L, mask_block=32) == b.ENTMAX_ERR_UNSUPPORTED      # bf16 path uses 64
     assert _fwd(L, bins=100) == b.ENTMAX_ERR_UNSUPPORTED
