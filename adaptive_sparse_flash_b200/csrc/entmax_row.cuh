@@ -235,8 +235,10 @@ __device__ __forceinline__ void stash_sums(const Stash& st, const float* stash, 
 // For k = 1 and k = 2 the root is found in closed form on its segment (exact integer moments); for
 // other k by a search over the bin edges and then bisection inside the segment, keeping the end where
 // f >= 0. T[i] = i^k for i = 0..B (generic k only). The result is lowered by a few float32 ulps so that
-// rounding cannot lift it above the binned root.
-template <int KIND>
+// rounding cannot lift it above the binned root. I is the integer type of the moments: int is exact while
+// the row holds at most a few hundred entries (every moment stays below 2^31 before the crossing: A0 <= 2^9,
+// offsets <= 2^9), long long for any count.
+template <int KIND, typename I = long long>
 __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, const uint16_t* hist, int r, const float* T) {
     const int B = sp.bins;
     auto cnt = [&](int j) -> uint32_t {
@@ -249,12 +251,12 @@ __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, cons
         // Only live bins are visited (set bits of the live mask, in order of offset j = top - bin); between
         // them the moments move in closed form, and the first J at which the binned function reaches 0
         // (A2 >= (B-1)^2, or A1 >= B-1 for k = 1) is found by a float estimate corrected in integers.
-        long long A0 = 0, A1 = 0, A2 = 0;
-        const long long thr = (KIND == kAlpha15) ? (long long)(B - 1) * (B - 1) : (long long)(B - 1);
-        auto Ak = [&](long long t) -> long long {  // A_k(J0 + t) from the moments at J0
+        I A0 = 0, A1 = 0, A2 = 0;
+        const I thr = (KIND == kAlpha15) ? (I)(B - 1) * (B - 1) : (I)(B - 1);
+        auto Ak = [&](I t) -> I {  // A_k(J0 + t) from the moments at J0
             return (KIND == kAlpha15) ? A2 + 2 * t * A1 + t * t * A0 : A1 + t * A0;
         };
-        auto first_cross = [&]() -> long long {  // smallest t >= 1 with A_k(J0 + t) >= thr (A0 > 0)
+        auto first_cross = [&]() -> I {  // smallest t >= 1 with A_k(J0 + t) >= thr (A0 > 0)
             float tf;
             if constexpr (KIND == kAlpha15) {
                 const float a0 = (float)A0, a1 = (float)A1, d2 = (float)(A2 - thr);
@@ -262,7 +264,7 @@ __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, cons
             } else {
                 tf = (float)(thr - A1) / (float)A0;
             }
-            long long t = (long long)fmaxf(1.0f, ceilf(tf));
+            I t = (I)fmaxf(1.0f, ceilf(tf));
             while (t > 1 && Ak(t - 1) >= thr) --t;
             while (Ak(t) < thr) ++t;
             return t;
@@ -286,16 +288,16 @@ __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, cons
 #endif
                 bits &= ~(1u << bpos);
                 const int sl = wi * 32 + bpos;
-                const long long c = hist[sl * kTileRows + r];
+                const I c = hist[sl * kTileRows + r];
                 if (c == 0) continue;
                 const int jn = (stop - sl) & (B - 1);  // offset of this bin below the top
                 const int J1 = jn + 1;                 // first J at which the bin counts
                 if (A0 > 0) {
-                    const long long T = J1 - J0;
+                    const I T = J1 - J0;
                     // crosses before this bin starts to count iff A_k(J1 - 1) reaches thr (A_k is
                     // nondecreasing in J); only then is the crossing located
                     if (T >= 2 && Ak(T - 1) >= thr) {
-                        const long long t = first_cross();
+                        const I t = first_cross();
                         A2 = (KIND == kAlpha15) ? Ak(t) : A2;
                         A1 += t * A0;
                         J = J0 + (int)t;
@@ -313,7 +315,7 @@ __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, cons
             }
         }
         if (!found && A0 > 0) {
-            const long long t = first_cross();
+            const I t = first_cross();
             A2 = (KIND == kAlpha15) ? Ak(t) : A2;
             A1 += t * A0;
             J = J0 + (int)t;

@@ -113,7 +113,9 @@ enum : int {
     kXF0 = 7, kXF1 = 8, kXF2 = 9, kXF0b = 10,    // partial sums of warpgroup 1
     kXOvf = 11,                                  // 1: the row's candidates did not fit the stash
     kXCnt = 12,                                  // partial support count of warpgroup 1 (int bits)
-    kXRows = 13
+    kXRows = 13,
+    kXCnt0 = kXF0b                               // warpgroup 0: stash count (int bits), -1 when its half
+                                                 // overflowed; only between the dense sweep and the solve
 };
 
 struct Small {
@@ -174,15 +176,6 @@ __device__ __forceinline__ void hist_start(HistRow& h, float m_raw, const SolveP
     h.m_raw = m_raw;
     h.thr_raw = m_raw - sp.inv_cz;
     h.top = h.any ? bin_of(m_raw, sp.cbin) : 0;
-}
-
-// Bin the entries of one stash half above the row's threshold.
-static __device__ __noinline__ void hist_bin_half(HistRow& h, const float* st, int n, const SolveParams& sp,
-                                                  uint16_t* hist, int r) {
-    for (int i = 0; i < n; ++i) {
-        const float v = st[i * BM + r];
-        if (v > h.thr_raw) hist_add(h, v, sp.cbin, sp.bins, hist, r);
-    }
 }
 
 // Bin the entries above the threshold of one staged block (rb[c * 128], c < 64; rb points at the row), groups
@@ -591,8 +584,42 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0 && ball) atomicOr(&next[J >> 5], 1u << (J & 31));
         }
         lcs += nblk;
-        if (g == 1) sm.xf[kXCnt1][r] = __int_as_float(ovf ? -1 : nst);
+        sm.xf[g ? kXCnt1 : kXCnt0][r] = __int_as_float(ovf ? -1 : nst);
         ok = !bar_or256(!ok || *abort_flag != 0);
+
+        // ---- the rows' histograms, binned from both stash halves at once (window fixed by the final max) ----
+        // Counts are u16 [slot][128]; the two warpgroups' threads of a row add into it with 32-bit shared
+        // atomics on the word holding the row's count (a count stays below 2^16, so the neighbouring row's
+        // half-word is untouched) and set the slot's live bit with an atomic OR.
+        {
+            const float m_fin = fmaxf(sm.xf[kXMax0][r], sm.xf[kXMax1][r]);
+            const bool binit = ok && valid && sp.init_mode == 0 && __float_as_int(sm.xf[kXCnt0][r]) >= 0 &&
+                               __float_as_int(sm.xf[kXCnt1][r]) >= 0;
+            uint32_t* hist32 = reinterpret_cast<uint32_t*>(hist);
+            for (int i = tid; i < NB * BM / 2; i += kCompute) hist32[i] = 0u;
+            uint32_t* live_r = live_all + r * HC::kStride;
+            if (g == 0)
+                for (int i = 0; i < HC::kStride - 1; ++i) live_r[i] = 0u;
+            named_bar_sync(1, kCompute);
+            if (binit) {
+                const int top = bin_of(m_fin, sp.cbin);
+                const float thr_raw = m_fin - sp.inv_cz;
+                const uint32_t inc = 1u << (16 * (r & 1));
+                for (int i = 0; i < nst; ++i) {
+                    const float v = st_mine[i * BM + r];
+                    if (v > thr_raw) {
+                        const int b = bin_of(v, sp.cbin);
+                        const int j = top - b;
+                        if (j >= 0 && j < sp.bins) {
+                            const int sl = b & (sp.bins - 1);
+                            atomicAdd(&hist32[(sl * BM + r) >> 1], inc);
+                            atomicOr(&live_r[sl >> 5], 1u << (sl & 31));
+                        }
+                    }
+                }
+            }
+            named_bar_sync(1, kCompute);
+        }
 
         // ---- per-row solve (warpgroup 0 owns the solver state of its row) ----
         HistRow h;
@@ -603,7 +630,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         float m_raw = -INFINITY;
         int n1 = 0;
         if (g == 0) {
-            hist_init(h, live_all, r, HC::kStride);
+            // the live words were cleared and set by the binning above
+            h.nlw = HC::kStride - 1;
+            h.live = live_all + r * HC::kStride;
             const int c1 = __float_as_int(sm.xf[kXCnt1][r]);
             m_raw = fmaxf(m_run, sm.xf[kXMax1][r]);
             row_ovf = ovf || c1 < 0;
@@ -611,10 +640,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float m = sp.cz * m_raw;
             float tau_h = m - 1.0f;
             if (ok && valid && !row_ovf && sp.init_mode == 0) {
-                hist_start(h, m_raw, sp);
-                hist_bin_half(h, st_mine, nst, sp, hist, r);
-                hist_bin_half(h, stash + kHalf * BM, n1, sp, hist, r);
-                tau_h = hist_tau<KIND>(h, sp, hist, r, sm.T);
+                // the window and the counts are in place (binned above); at most 2 kHalf entries per row, so
+                // 32-bit moments are exact
+                h.any = m_raw > -INFINITY;
+                h.m_raw = m_raw;
+                h.thr_raw = m_raw - sp.inv_cz;
+                h.top = h.any ? bin_of(m_raw, sp.cbin) : 0;
+                tau_h = hist_tau<KIND, int>(h, sp, hist, r, sm.T);
             }
             solve_init(s, valid ? tau_h : 0.0f, valid ? m : 1.0f, n_i, sp);
             if (!valid) s.done = true;
@@ -946,7 +978,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int nh = elem_cnt[hh * BM + r];
                     const uint16_t* kk = elem_key + hh * (kCap * BM) + r;
                     const float* pk = elem_p + hh * (kCap * BM) + r;
-#pragma unroll 2
+#pragma unroll 4
                     for (int e = 0; e < nh; ++e) {
                         const uint4* src = reinterpret_cast<const uint4*>(Vh + (size_t)kk[e * BM] * D);
                         const float pe = pk[e * BM];
