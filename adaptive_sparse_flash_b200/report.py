@@ -212,6 +212,21 @@ def timing_report(out=sys.stdout):
     print(f"| workload | alpha | pass | entmax fwd ms | entmax bwd ms | effective TFLOP/s | frac of bf16 burst "
           f"({peak:g}, {src}) | dense fwd (+bwd) ms | block sparsity |", file=out)
     print("|---|---|---|---|---|---|---|---|---|", file=out)
+    # cfg1: fp32 inputs, non-causal, mask blocks of 32 (the FMA kernel; the dense baseline takes bf16 only)
+    import numpy as np
+    from . import inputs as inp
+    arr = inp.iid(1, 1, 256, 64, seed=0, beta=1.0, dtype="fp32", with_dO=False)
+    Q1, K1, V1 = (torch.from_numpy(np.ascontiguousarray(arr[k])).cuda() for k in ("Q", "K", "V"))
+    ws1 = b.alloc_workspace(1, 1, 256, 64, b.ENTMAX_FP32, opts=b.make_opts(mask_block=32))
+    o1 = b.make_opts(ws1, mask_block=32)
+    O1 = torch.empty_like(Q1)
+    t1 = torch.empty((1, 1, 256), dtype=torch.float32, device="cuda")
+    m1 = torch.empty(b.mask_shape(1, 1, 256, 32), dtype=torch.int32, device="cuda")
+    f1 = timed(lambda: b.entmax_attn_fwd(Q1, K1, V1, O1, t1, m1, 1.5, False, o1))
+    nnz1 = int(np.unpackbits(m1.cpu().numpy().view(np.uint8), bitorder="little").sum())
+    fl1 = 2.0 * 64 * 256 * 256 + 2.0 * 64 * 32 * 32 * nnz1
+    print(f"| cfg1 B=1 H=1 n=256 d=64 fp32 non-causal | 1.5 | fwd | {f1:.3f} | - | {fl1 / (f1 * 1e-3) / 1e12:.2f} | "
+          f"{fl1 / (f1 * 1e-3) / 1e12 / peak:.4f} | - | {1 - nnz1 / 64:.3f} |", file=out, flush=True)
     for name, kind, B, H, n, d, alphas, psets in CONFIGS:
         for params in psets:
             arr = _gen(kind, B, H, n, d, params)

@@ -6,7 +6,7 @@ One step = entmax_attn_fwd + entmax_attn_bwd over one batch of the long-context 
 dense Q K^T pass over the causal entries plus the P V and backward products of the nonzero
 64 x 64 mask blocks only:  2 d n(n+1)/2 + (2 + 5 * 2) d 64 64 N_nz  per head.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-sweep] [--no-cpu]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--no-sweep] [--no-cpu] [--oracle-table]
 
 Prints one JSON line (rank 0). Under torchrun each rank runs its own copy of the workload (independent
 heads: no data-path collective), times on its device, and the max over ranks is reported.
@@ -262,6 +262,40 @@ def cpu_baseline(arr):
                       f"{sec:.1f} s, scaled by that head's effective FLOPs", "seconds": sec}
 
 
+# (label, generator kind, B, H, n, d, alpha, params, causal, backward): one row per configuration of the
+# parity tests, for the oracle's per-configuration CPU time
+ORACLE_TABLE = (
+    ("cfg1 1x1x256x64 fp32 non-causal", "iid", 1, 1, 256, 64, 1.5, {"beta": 1.0}, False, False),
+    ("cfg2 4x8x1024x64 beta=4", "iid", 4, 8, 1024, 64, 1.5, {"beta": 4.0}, True, False),
+    ("cfg3 2x16x4096x128 beta=8", "iid", 2, 16, 4096, 128, 1.5, {"beta": 8.0}, True, True),
+    ("cfg4 1x16x16384x64 clustered", "clustered", 1, 16, 16384, 64, 1.5, {"centres": 256, "beta_q": 6.0}, True, True),
+    ("cfg5 8x12x2048x64 clustered beta_q=4", "clustered", 8, 12, 2048, 64, 1.5, {"centres": 64, "beta_q": 4.0}, True, True),
+)
+
+
+def oracle_table():
+    """The float64 oracle's CPU time per configuration: one head timed (forward, and backward where the
+    configuration has one), scaled to the configuration's heads. Prints a markdown table."""
+    from adaptive_sparse_flash_b200 import inputs as _inputs
+    from oracle import attention as oa
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    print(f"| configuration | oracle s, one head | heads | oracle s, whole configuration ({cores} cores) |")
+    print("|---|---|---|---|")
+    for label, kind, Bc, Hc, n, d, alpha, params, causal, bwd in ORACLE_TABLE:
+        if kind == "iid":
+            arr = _inputs.iid(1, 1, n, d, seed=0, beta=params["beta"], dtype="fp32" if "fp32" in label else "bf16",
+                              with_dO=bwd)
+        else:
+            arr = _inputs.clustered(1, 1, n, d, centres=params["centres"], beta_q=params["beta_q"], seed=0)
+        t0 = time.perf_counter()
+        oa.forward(arr["Q"], arr["K"], arr["V"], alpha, causal)
+        if bwd:
+            oa.backward(arr["Q"], arr["K"], arr["V"], arr["dO"], alpha, causal)
+        sec = time.perf_counter() - t0
+        print(f"| {label} ({'fwd+bwd' if bwd else 'fwd'}) | {sec:.2f} | {Bc * Hc} | {sec * Bc * Hc:.1f} |", flush=True)
+    return 0
+
+
 def rank_env():
     """(rank, world size, local rank) from the launcher's environment; one process per GPU."""
     return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
@@ -358,7 +392,11 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-sweep", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--oracle-table", action="store_true",
+                    help="print the float64 oracle's CPU time per configuration and exit (no GPU)")
     args = ap.parse_args()
+    if args.oracle_table:
+        return oracle_table()
     if args.warmup < 3:
         args.warmup = 3
 
