@@ -241,10 +241,6 @@ __device__ __forceinline__ void stash_sums(const Stash& st, const float* stash, 
 template <int KIND, typename I = long long>
 __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, const uint16_t* hist, int r, const float* T) {
     const int B = sp.bins;
-    auto cnt = [&](int j) -> uint32_t {
-        const int sl = (h.top - j) & (B - 1);
-        return ((h.live[sl >> 5] >> (sl & 31)) & 1u) ? (uint32_t)hist[sl * kTileRows + r] : 0u;
-    };
     float tau_h;
     if constexpr (KIND == kAlpha15 || KIND == kAlpha2) {
         // A0 = sum c_j, A1 = sum c_j (J - j), A2 = sum c_j (J - j)^2 over offsets j < J (exact integers).
@@ -333,12 +329,35 @@ __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, cons
         tau_h = ((float)(h.top - J) + u) * sp.w;
     } else {
         const float thr = T[B - 1];
+        // visit the nonzero bins at offsets j < J in ascending j (live slots stop, stop - 1, ..., 0, B - 1, ...,
+        // stop + 1, word by word), so that each evaluation costs the row's nonzero bins, not J
+        const int stop = h.top & (B - 1);
+        const int nw = B >= 32 ? B / 32 : 1;
+        auto for_nonzero = [&](int J, auto&& fn) {
+            for (int step = 0; step <= nw; ++step) {
+                const int wi = ((stop >> 5) - step + 2 * nw) % nw;
+                uint32_t bits = h.live[wi];
+                if (B < 32) bits &= (1u << B) - 1u;
+                if (step == 0) bits &= (stop & 31) == 31 ? 0xffffffffu : ((2u << (stop & 31)) - 1u);
+                if (step == nw) bits &= (stop & 31) == 31 ? 0u : ~((2u << (stop & 31)) - 1u);
+                while (bits) {
+#ifdef __CUDA_ARCH__
+                    const int bpos = 31 - __clz(bits);
+#else
+                    const int bpos = 31 - __builtin_clz(bits);
+#endif
+                    bits &= ~(1u << bpos);
+                    const int sl = wi * 32 + bpos;
+                    const int j = (stop - sl) & (B - 1);
+                    if (j >= J) return;
+                    const uint32_t c = hist[sl * kTileRows + r];
+                    if (c) fn(j, c);
+                }
+            }
+        };
         auto F = [&](int J) -> float {
             float s = 0.0f;
-            for (int j = 0; j < J; ++j) {
-                const uint32_t c = cnt(j);
-                if (c) s = fmaf((float)c, T[J - j], s);
-            }
+            for_nonzero(J, [&](int j, uint32_t c) { s = fmaf((float)c, T[J - j], s); });
             return s;
         };
         // smallest J in [1, B-1] with F(J) >= thr (F is nondecreasing in J)
@@ -353,15 +372,14 @@ __host__ __device__ float hist_tau(const HistRow& h, const SolveParams& sp, cons
         for (int it = 0; it < 6; ++it) {
             const float um = 0.5f * (ulo + uhi);
             float s = 0.0f;
-            for (int j = 0; j < J; ++j) {
-                const uint32_t c = cnt(j);
+            for_nonzero(J, [&](int j, uint32_t c) {
                 const float x = (float)(J - j) - um;
 #ifdef __CUDA_ARCH__
-                if (c && x > 0.0f) s = fmaf((float)c, exp2f(sp.k * __log2f(x)), s);
+                if (x > 0.0f) s = fmaf((float)c, exp2f(sp.k * __log2f(x)), s);
 #else
-                if (c && x > 0.0f) s = fmaf((float)c, exp2f(sp.k * log2f(x)), s);
+                if (x > 0.0f) s = fmaf((float)c, exp2f(sp.k * log2f(x)), s);
 #endif
-            }
+            });
             if (s >= thr) ulo = um; else uhi = um;
         }
         tau_h = ((float)(h.top - J) + ulo) * sp.w;
