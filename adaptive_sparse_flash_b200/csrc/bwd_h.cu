@@ -60,7 +60,6 @@ constexpr uint64_t kDescK = sdesc_sw128_fields(16, 1024);
 constexpr uint64_t kDescMN = sdesc_sw128_fields(64 * 128, 1024);
 
 constexpr int kThreads = 352;
-constexpr int kCompute = 256;
 constexpr int TM = 128;  // rows of the CTA's tile
 constexpr int TB = 64;   // rows of a walked block
 constexpr int D = 64;
@@ -716,51 +715,50 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if constexpr (delta_only) {
 #pragma unroll
                     for (int c = 0; c < TB; ++c) rs = fmaf(sv[c], dp[c], rs);
-                    ++j;
-                    continue;
-                }
-#pragma unroll
-                for (int c = 0; c < TB; ++c) {
-                    const float e = sv[c] * (dp[c] - dl);
-                    if (ab) rs += e;
-                    dp[c] = e * sc.ds;
-                }
-                ok = __all_sync(0xffffffffu, wait_bounded(&bb.a_empty[g], (j & 1) ^ 1, abort_flag, a.status));
-                if (!ok) break;
-                const uint32_t ta = lane_base + 256u + 64u * g;
-                if (ab) {
-                    // [u g | u], one fp16 term each (keys of unit scale), 32 keys at a time
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t wa[16], wu[16];
-#pragma unroll
-                        for (int c = 0; c < 32; c += 2) {
-                            wa[c / 2] = pack_half2(dp[32 * h + c], dp[32 * h + c + 1]);
-                            wu[c / 2] = pack_half2(sv[32 * h + c], sv[32 * h + c + 1]);
-                        }
-                        tmem_st16(ta + 16 * h, wa);
-                        tmem_st16(ta + 32 + 16 * h, wu);
-                    }
-                } else if (one) {
-                    uint32_t w32[32];
-#pragma unroll
-                    for (int c = 0; c < TB; c += 2) w32[c / 2] = pack_half2(dp[c], dp[c + 1]);
-                    tmem_st32(ta, w32);
                 } else {
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        uint32_t whi[16], wlo[16];
-#pragma unroll
-                        for (int c = 0; c < 32; c += 2)
-                            split_half2(dp[32 * h + c], dp[32 * h + c + 1], whi[c / 2], wlo[c / 2]);
-                        tmem_st16(ta + 16 * h, whi);
-                        tmem_st16(ta + 32 + 16 * h, wlo);
+                    for (int c = 0; c < TB; ++c) {
+                        const float e = sv[c] * (dp[c] - dl);
+                        if (ab) rs += e;
+                        dp[c] = e * sc.ds;
                     }
+                    ok = __all_sync(0xffffffffu, wait_bounded(&bb.a_empty[g], (j & 1) ^ 1, abort_flag, a.status));
+                    if (!ok) break;
+                    const uint32_t ta = lane_base + 256u + 64u * g;
+                    if (ab) {
+                        // [u g | u], one fp16 term each (keys of unit scale), 32 keys at a time
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t wa[16], wu[16];
+#pragma unroll
+                            for (int c = 0; c < 32; c += 2) {
+                                wa[c / 2] = pack_half2(dp[32 * h + c], dp[32 * h + c + 1]);
+                                wu[c / 2] = pack_half2(sv[32 * h + c], sv[32 * h + c + 1]);
+                            }
+                            tmem_st16(ta + 16 * h, wa);
+                            tmem_st16(ta + 32 + 16 * h, wu);
+                        }
+                    } else if (one) {
+                        uint32_t w32[32];
+#pragma unroll
+                        for (int c = 0; c < TB; c += 2) w32[c / 2] = pack_half2(dp[c], dp[c + 1]);
+                        tmem_st32(ta, w32);
+                    } else {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t whi[16], wlo[16];
+#pragma unroll
+                            for (int c = 0; c < 32; c += 2)
+                                split_half2(dp[32 * h + c], dp[32 * h + c + 1], whi[c / 2], wlo[c / 2]);
+                            tmem_st16(ta + 16 * h, whi);
+                            tmem_st16(ta + 32 + 16 * h, wlo);
+                        }
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bb.a_full[g]);
                 }
-                tmem_st_wait();
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bb.a_full[g]);
                 ++j;
             }
         }
