@@ -30,8 +30,9 @@
 // Sweeps follow the plan protocol of the bf16 forward (fwd_tc.cu): before each sweep the compute warps
 // publish its kind and its set of key blocks, which the issuing warps follow.
 //   dense   - every causal key block: running max and the candidate stash (entries above max - 1); the
-//             stash of a row has one half per warpgroup. The row's histogram is binned from the stash
-//             when the sweep ends and its tau is solved on chip from the stash.
+//             stash of a row has one half per warpgroup. When the sweep ends both warpgroups bin their
+//             halves into the row's histogram (window at the final max), and warpgroup 0 takes tau_h and
+//             solves tau on chip from the stash.
 //   hist    - only when some row's stash half overflowed: candidate blocks, all on warpgroup 0, which
 //             bins those rows' entries into their histograms with the window fixed by the final max;
 //   refine  - candidate blocks: solver sums at the current tau (partial sums of the two warpgroups are
