@@ -16,8 +16,8 @@
  * bit-packed mask, 32 key blocks per uint32 ("Bit-Packed Block Mask"), and computes P V only on those
  * blocks (or, where every row of a 128-row tile was solved on chip and has a small support, as a sum over
  * the support entries gathered from V in fp32). The backward walks the same mask ("GPU-Optimierung":
- * find-next-set and popcount over the
- * nonzero blocks) with the entmax Jacobian dS = u (g - delta), u = p^(2 - alpha) on the support,
+ * find-next-set and popcount over the nonzero blocks) with the entmax Jacobian dS = u (g - delta),
+ * u = p^(2 - alpha) on the support,
  * g = dO V^T, delta = sum(u g) / sum(u).
  *
  * Conventions for every entry point
