@@ -17,8 +17,7 @@
  * blocks (or, where every row of a 128-row tile was solved on chip and has a small support, as a sum over
  * the support entries gathered from V in fp32). The backward walks the same mask ("GPU-Optimierung":
  * find-next-set and popcount over the nonzero blocks) with the entmax Jacobian dS = u (g - delta),
- * u = p^(2 - alpha) on the support,
- * g = dO V^T, delta = sum(u g) / sum(u).
+ * u = p^(2 - alpha) on the support, g = dO V^T, delta = sum(u g) / sum(u).
  *
  * Conventions for every entry point
  *   - Tensors are [B, H, n, d] row-major, d fastest, on the current CUDA device. bf16 tensors use
